@@ -1,0 +1,323 @@
+/*
+ * msa_oracle.c -- plain CPU oracle for the MiniMax Sparse Attention (MSA) forward path.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path may call, link or load this file;
+ * only the tests, the package's smoke check and the benchmark's CPU-baseline leg use it.
+ * It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes is the method's plain definition, in double precision, with no blocking,
+ * fusion or reordering beyond the definition:
+ *
+ *  (1) Index Branch (MSA explainer "MiniMax Sparse Attention", Figure 1 and section 05-1;
+ *      paper abstract): for query row i and GQA group r, score every visible key j <= i with
+ *      s_j = q_idx[i,r] . k_idx[j,r]; max-pool the scores over each B_k-token KV block; pick
+ *      the Top-k blocks per (i, r) on the raw scores (softmax keeps the order, so no exp is
+ *      needed), always keeping the local block floor(i/B_k), which counts toward k.
+ *      Readings where the pages are silent: ties go to the lower block index; a block b is
+ *      visible iff b*B_k <= i; the selected set is emitted ascending, padded with -1; its size
+ *      is min(k, floor(i/B_k)+1).
+ *  (2) KV->Q inversion (explainer section 05-2, "KV-outer" paragraph): for every (r, b) the
+ *      ascending list of query rows i whose set contains b, each entry i*k + slot where slot is
+ *      the rank of b in i's ascending set.
+ *  (3) Main Branch (explainer sections 02 and 05-2; abstract "exact block-sparse attention"):
+ *      exact softmax attention of head h (group r = floor(h/G), adjacent heads share a KV head,
+ *      explainer section 01) over the tokens T = {j <= i : j in a selected block}, logits
+ *      q_h . k_j / sqrt(d_h); out = sum_j p_j v_j; lse = max + log(sum exp(. - max)) in the
+ *      units of the scaled logits.
+ *  (4) Decode: (1)+(3) for the single query at position len-1 of each cached sequence.
+ *
+ * Inputs are bf16 bit patterns widened exactly to double. All sums are in double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static inline double bf16_to_double(uint16_t x)
+{
+    uint32_t u = (uint32_t)x << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static void set_threads(int n_threads)
+{
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+}
+
+int msa_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* (1) Index Branch: score, block max-pool, Top-k with the forced local block.               */
+/* ---------------------------------------------------------------------------------------- */
+
+typedef struct {
+    double score;
+    int32_t block;
+} scored_block;
+
+/* Sort order of the Top-k: larger pooled score first; equal scores, lower block first. */
+static int by_score_then_block(const void* a, const void* b)
+{
+    const scored_block* x = (const scored_block*)a;
+    const scored_block* y = (const scored_block*)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->block > y->block) - (x->block < y->block);
+}
+
+static int ascending_int(const void* a, const void* b)
+{
+    int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+    return (x > y) - (x < y);
+}
+
+/*
+ * Selection for one query row of one group.
+ *   qrow : d_idx bf16 values of q_idx[i, r]
+ *   kseq : k_idx of the sequence, element (j, r, d) at kseq[(j*H_kv + r)*d_idx + d]
+ *   i    : query position
+ *   sel  : k outputs
+ *   work : scratch of at least floor(i/B_k) entries
+ */
+static void select_one(const uint16_t* qrow, const uint16_t* kseq, int64_t i, int r, int H_kv, int d_idx,
+                       int B_k, int k, int32_t* sel, scored_block* work)
+{
+    const int64_t local = i / B_k;          /* the forced local block */
+    const int64_t n_candidates = local;     /* blocks 0 .. local-1 are fully visible */
+    double q[512];
+    for (int d = 0; d < d_idx; ++d) q[d] = bf16_to_double(qrow[d]);
+
+    for (int64_t b = 0; b < n_candidates; ++b) {
+        double best = -INFINITY;
+        for (int64_t j = b * B_k; j < (b + 1) * B_k; ++j) {
+            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_idx;
+            double s = 0.0;
+            for (int d = 0; d < d_idx; ++d) s += q[d] * bf16_to_double(kr[d]);
+            if (s > best) best = s; /* block max pooling */
+        }
+        work[b].score = best;
+        work[b].block = (int32_t)b;
+    }
+    qsort(work, (size_t)n_candidates, sizeof(scored_block), by_score_then_block);
+
+    int n = 0;
+    const int64_t take = n_candidates < (int64_t)(k - 1) ? n_candidates : (int64_t)(k - 1);
+    for (int64_t t = 0; t < take; ++t) sel[n++] = work[t].block;
+    sel[n++] = (int32_t)local;
+    qsort(sel, (size_t)n, sizeof(int32_t), ascending_int);
+    for (int t = n; t < k; ++t) sel[t] = -1;
+}
+
+/*
+ * Selections for a set of query rows of one sequence.
+ *   q_idx : [n_rows, H_kv, d_idx] bf16, the index queries of the requested rows (gathered)
+ *   rows  : [n_rows] positions i (each < N)
+ *   k_idx : [N, H_kv, d_idx] bf16
+ *   sel   : [n_rows, H_kv, k] int32 out
+ * Returns 0, or -1 on bad arguments.
+ */
+int msa_oracle_select_rows(const uint16_t* q_idx, const int64_t* rows, int64_t n_rows, const uint16_t* k_idx,
+                           int64_t N, int H_kv, int d_idx, int B_k, int k, int32_t* sel, int n_threads)
+{
+    if (!q_idx || !rows || !k_idx || !sel || N < 1 || H_kv < 1 || d_idx < 1 || d_idx > 512 || B_k < 1 || k < 1)
+        return -1;
+    for (int64_t t = 0; t < n_rows; ++t)
+        if (rows[t] < 0 || rows[t] >= N) return -1;
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        scored_block* work = (scored_block*)malloc(sizeof(scored_block) * (size_t)(N / B_k + 1));
+        if (!work) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1) collapse(2)
+        for (int64_t t = 0; t < n_rows; ++t)
+            for (int r = 0; r < H_kv; ++r)
+                if (work)
+                    select_one(q_idx + ((size_t)t * H_kv + r) * d_idx, k_idx, rows[t], r, H_kv, d_idx, B_k, k,
+                               sel + ((size_t)t * H_kv + r) * k, work);
+        free(work);
+    }
+    return err;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* (2) KV -> Q inversion.                                                                     */
+/* ---------------------------------------------------------------------------------------- */
+
+/*
+ *   block_idx : [H_kv, N, k] int32, ascending, -1 padded
+ *   offsets   : [H_kv, nb+1] int64 out, CSR row pointers per group (offsets[r][0] = 0)
+ *   entries   : [H_kv, N*k] int32 out, entries of group r start at entries + r*N*k
+ * For each (r, b) the entries are the rows i (ascending) whose set holds b, encoded i*k + slot.
+ * Returns 0, or -1 on an out-of-range block id.
+ */
+int msa_oracle_kv2q(const int32_t* block_idx, int64_t N, int H_kv, int B_k, int k, int64_t* offsets,
+                    int32_t* entries)
+{
+    const int64_t nb = (N + B_k - 1) / B_k;
+    for (int r = 0; r < H_kv; ++r) {
+        const int32_t* sel = block_idx + (size_t)r * N * k;
+        int64_t* off = offsets + (size_t)r * (nb + 1);
+        int32_t* ent = entries + (size_t)r * N * k;
+        for (int64_t b = 0; b <= nb; ++b) off[b] = 0;
+        for (int64_t i = 0; i < N; ++i)
+            for (int s = 0; s < k; ++s) {
+                int32_t b = sel[i * k + s];
+                if (b < 0) continue;
+                if (b >= nb) return -1;
+                off[b + 1] += 1;
+            }
+        for (int64_t b = 0; b < nb; ++b) off[b + 1] += off[b];
+        int64_t* fill = (int64_t*)malloc(sizeof(int64_t) * (size_t)nb);
+        if (!fill) return -1;
+        for (int64_t b = 0; b < nb; ++b) fill[b] = off[b];
+        for (int64_t i = 0; i < N; ++i) /* ascending i keeps each list sorted by row */
+            for (int s = 0; s < k; ++s) {
+                int32_t b = sel[i * k + s];
+                if (b < 0) continue;
+                ent[fill[b]++] = (int32_t)(i * k + s);
+            }
+        free(fill);
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* (3) Main Branch: exact softmax attention over the selected blocks' visible tokens.        */
+/* ---------------------------------------------------------------------------------------- */
+
+/*
+ * One (row, head).
+ *   qh   : d_h bf16, q[i, h]
+ *   kseq, vseq : [*, H_kv, d_h] bf16 of the sequence
+ *   sel  : k block ids of (i, r), -1 padded
+ *   out  : d_h doubles; *lse out
+ *   logits : scratch of k*B_k doubles
+ */
+static void attend_one(const uint16_t* qh, const uint16_t* kseq, const uint16_t* vseq, int64_t i, int r, int H_kv,
+                       int d_h, int B_k, int k, const int32_t* sel, double* out, double* lse, double* logits)
+{
+    const double scale = 1.0 / sqrt((double)d_h);
+    double q[512];
+    for (int d = 0; d < d_h; ++d) q[d] = bf16_to_double(qh[d]);
+
+    /* logits over T, in the order of the selected blocks */
+    int64_t n = 0;
+    double m = -INFINITY;
+    for (int s = 0; s < k; ++s) {
+        int32_t b = sel[s];
+        if (b < 0) continue;
+        for (int64_t j = (int64_t)b * B_k; j < ((int64_t)b + 1) * B_k && j <= i; ++j) {
+            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;
+            double dot = 0.0;
+            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);
+            logits[n] = dot * scale;
+            if (logits[n] > m) m = logits[n];
+            ++n;
+        }
+    }
+    double z = 0.0;
+    for (int d = 0; d < d_h; ++d) out[d] = 0.0;
+    n = 0;
+    for (int s = 0; s < k; ++s) {
+        int32_t b = sel[s];
+        if (b < 0) continue;
+        for (int64_t j = (int64_t)b * B_k; j < ((int64_t)b + 1) * B_k && j <= i; ++j) {
+            double p = exp(logits[n++] - m);
+            z += p;
+            const uint16_t* vr = vseq + ((size_t)j * H_kv + r) * d_h;
+            for (int d = 0; d < d_h; ++d) out[d] += p * bf16_to_double(vr[d]);
+        }
+    }
+    for (int d = 0; d < d_h; ++d) out[d] /= z;
+    *lse = m + log(z);
+}
+
+/*
+ *   q    : [n_rows, H_q, d_h] bf16, the requested rows' queries (gathered)
+ *   rows : [n_rows] positions
+ *   kk, v: [N, H_kv, d_h] bf16
+ *   sel  : [n_rows, H_kv, k] int32 (from msa_oracle_select_rows)
+ *   out  : [n_rows, H_q, d_h] double; lse : [n_rows, H_q] double
+ */
+int msa_oracle_attend_rows(const uint16_t* q, const int64_t* rows, int64_t n_rows, const uint16_t* kk,
+                           const uint16_t* v, int64_t N, int H_q, int H_kv, int d_h, int B_k, int k,
+                           const int32_t* sel, double* out, double* lse, int n_threads)
+{
+    if (!q || !rows || !kk || !v || !sel || !out || !lse || H_kv < 1 || H_q % H_kv || d_h < 1 || d_h > 512)
+        return -1;
+    for (int64_t t = 0; t < n_rows; ++t)
+        if (rows[t] < 0 || rows[t] >= N) return -1;
+    const int G = H_q / H_kv;
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        double* logits = (double*)malloc(sizeof(double) * (size_t)k * B_k);
+        if (!logits) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1) collapse(2)
+        for (int64_t t = 0; t < n_rows; ++t)
+            for (int h = 0; h < H_q; ++h)
+                if (logits) {
+                    const int r = h / G;
+                    attend_one(q + ((size_t)t * H_q + h) * d_h, kk, v, rows[t], r, H_kv, d_h, B_k, k,
+                               sel + ((size_t)t * H_kv + r) * k, out + ((size_t)t * H_q + h) * d_h,
+                               lse + (size_t)t * H_q + h, logits);
+                }
+        free(logits);
+    }
+    return err;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* (4) Decode: one query per cached sequence, at position len-1.                              */
+/* ---------------------------------------------------------------------------------------- */
+
+/*
+ *   q      : [B, H_q, d_h] bf16;  q_idx : [B, H_kv, d_idx] bf16
+ *   k_cache, v_cache : [B, L_max, H_kv, d_h] bf16;  k_idx_cache : [B, L_max, H_kv, d_idx] bf16
+ *   lens   : [B] int32, 1 <= len <= L_max (the cache holds the current token)
+ *   out    : [B, H_q, d_h] double; lse : [B, H_q] double; sel : [B, H_kv, k] int32
+ */
+int msa_oracle_decode(const uint16_t* q, const uint16_t* q_idx, const uint16_t* k_cache, const uint16_t* v_cache,
+                      const uint16_t* k_idx_cache, const int32_t* lens, int B, int64_t L_max, int H_q, int H_kv,
+                      int d_h, int d_idx, int B_k, int k, double* out, double* lse, int32_t* sel, int n_threads)
+{
+    for (int beta = 0; beta < B; ++beta)
+        if (lens[beta] < 1 || lens[beta] > L_max) return -1;
+    for (int beta = 0; beta < B; ++beta) {
+        const int64_t row = lens[beta] - 1;
+        const size_t kv_off = (size_t)beta * L_max * H_kv * d_h;
+        const size_t ki_off = (size_t)beta * L_max * H_kv * d_idx;
+        int rc = msa_oracle_select_rows(q_idx + (size_t)beta * H_kv * d_idx, &row, 1, k_idx_cache + ki_off,
+                                        lens[beta], H_kv, d_idx, B_k, k, sel + (size_t)beta * H_kv * k, n_threads);
+        if (rc) return rc;
+        rc = msa_oracle_attend_rows(q + (size_t)beta * H_q * d_h, &row, 1, k_cache + kv_off, v_cache + kv_off,
+                                    lens[beta], H_q, H_kv, d_h, B_k, k, sel + (size_t)beta * H_kv * k,
+                                    out + (size_t)beta * H_q * d_h, lse + (size_t)beta * H_q, n_threads);
+        if (rc) return rc;
+    }
+    return 0;
+}

@@ -1,0 +1,264 @@
+"""Pin checks for the CPU oracle.
+
+Each check takes an ``oracle.Oracle`` instance and raises AssertionError on a mismatch. They
+pin the oracle to things other than itself: a dense brute force on tiny inputs, closed forms,
+textbook dense attention when the budget covers the whole context, invariants of the selected
+sets, and the split-then-merge identity. ``test_oracle_pins`` runs them on the real oracle and
+``test_oracle_mutants`` shows that each plausible mistake planted in a copy of the oracle fails
+at least one of them.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from block_sparse_long_idx_b200.synth import bf16_bits_to_f64, f32_to_bf16_bits, int_uniform_bf16, normal_bf16
+from tests import ref_numpy as ref
+
+# (N, H_q, H_kv, d_h, d_idx, B_k, k) -- small shapes spanning several blocks, ragged tails, k larger
+# than the number of visible blocks, G = 1 and G > 1.
+SEL_SHAPES = [
+    (1, 2, 1, 8, 4, 4, 2),
+    (37, 4, 2, 8, 8, 4, 3),
+    (64, 2, 2, 8, 16, 8, 4),
+    (130, 4, 1, 16, 8, 16, 5),
+    (300, 8, 2, 8, 32, 16, 8),
+    (517, 2, 1, 8, 8, 32, 4),
+]
+
+
+def _idx_inputs(N, H_kv, d_idx, seed, integer=True):
+    shp = (N, H_kv, d_idx)
+    if integer:
+        return int_uniform_bf16(shp, -3, 3, seed, "pq"), int_uniform_bf16(shp, -3, 3, seed, "pk")
+    return normal_bf16(shp, seed, "pq"), normal_bf16(shp, seed, "pk")
+
+
+def check_selection_bruteforce(o):
+    """Selection equals the dense brute force exactly (integer and non-integer index inputs)."""
+    for t, (N, _, H_kv, _, d_idx, B_k, k) in enumerate(SEL_SHAPES):
+        for integer in (True, False):
+            qi, ki = _idx_inputs(N, H_kv, d_idx, 100 + t, integer)
+            got = o.select_all(qi, ki, B_k, k)
+            want = ref.dense_selection(qi, ki, B_k, k)
+            assert np.array_equal(got, want), f"selection mismatch at shape {t} integer={integer}"
+
+
+def check_selection_ties_closed_form(o):
+    """q_idx == 0 makes every score 0: the set is the lowest k-1 visible blocks plus the local block."""
+    N, H_kv, d_idx, B_k, k = 200, 2, 8, 8, 5
+    qi = np.zeros((N, H_kv, d_idx), dtype=np.uint16)  # +0.0 in bf16
+    ki = int_uniform_bf16((N, H_kv, d_idx), -3, 3, 7, "tk")
+    got = o.select_all(qi, ki, B_k, k)
+    for i in range(N):
+        loc = i // B_k
+        want = sorted(set(range(min(k - 1, loc))) | {loc})
+        want = want + [-1] * (k - len(want))
+        for r in range(H_kv):
+            assert list(got[r, i]) == want, (i, r, list(got[r, i]), want)
+
+
+def check_selection_planted_winners(o):
+    """Blocks with k_idx = +3 (winners) beat blocks with k_idx = 0 when q_idx = +1; ties go lower."""
+    N, H_kv, d_idx, B_k, k = 256, 1, 4, 8, 4
+    nb = N // B_k
+    winners = {3, 5, 6, 11, 17, 18, 25, 30}
+    qi = f32_to_bf16_bits(np.ones((N, H_kv, d_idx), dtype=np.float32))
+    kf = np.zeros((N, H_kv, d_idx), dtype=np.float32)
+    for b in winners:
+        kf[b * B_k:(b + 1) * B_k] = 3.0
+    ki = f32_to_bf16_bits(kf)
+    got = o.select_all(qi, ki, B_k, k)[0]
+    for i in range(N):
+        loc = i // B_k
+        vis_w = [b for b in sorted(winners) if b < loc]
+        vis_o = [b for b in range(loc) if b not in winners]
+        pick = (vis_w + vis_o)[: k - 1]
+        want = sorted(pick + [loc])
+        want = want + [-1] * (k - len(want))
+        assert list(got[i]) == want, (i, list(got[i]), want)
+    assert nb == 32
+
+
+def check_selection_invariants(o):
+    """Local block kept, |set| = min(k, local+1), ascending, distinct, visible, -1 padding last."""
+    N, H_kv, d_idx, B_k, k = 700, 2, 16, 16, 6
+    qi, ki = _idx_inputs(N, H_kv, d_idx, 11)
+    sel = o.select_all(qi, ki, B_k, k)
+    for r in range(H_kv):
+        for i in range(N):
+            s = list(sel[r, i])
+            loc = i // B_k
+            n = min(k, loc + 1)
+            assert all(x >= 0 for x in s[:n]) and all(x == -1 for x in s[n:]), (r, i, s)
+            v = s[:n]
+            assert v == sorted(set(v)) and loc in v and max(v) == loc and min(v) >= 0, (r, i, s)
+
+
+def _attn_inputs(N, H_q, H_kv, d_h, d_idx, seed):
+    return {
+        "q": normal_bf16((N, H_q, d_h), seed, "aq"),
+        "k": normal_bf16((N, H_kv, d_h), seed, "ak"),
+        "v": normal_bf16((N, H_kv, d_h), seed, "av"),
+        "q_idx": int_uniform_bf16((N, H_kv, d_idx), -3, 3, seed, "aqi"),
+        "k_idx": int_uniform_bf16((N, H_kv, d_idx), -3, 3, seed, "aki"),
+    }
+
+
+def check_attention_dense_invariant(o):
+    """When k*B_k >= N every visible block is selected, so MSA equals dense causal GQA attention."""
+    for (N, H_q, H_kv, d_h, B_k, k) in [(64, 4, 2, 16, 16, 4), (100, 4, 1, 8, 8, 13), (96, 8, 2, 32, 32, 3)]:
+        inp = _attn_inputs(N, H_q, H_kv, d_h, 8, N)
+        rows = np.arange(N)
+        sel, out, lse = o.prefill_rows(inp, rows, B_k, k)
+        want, want_lse = ref.dense_causal_gqa(inp["q"], inp["k"], inp["v"])
+        assert np.max(np.abs(out - want)) < 1e-12, np.max(np.abs(out - want))
+        assert np.max(np.abs(lse - want_lse)) < 1e-12
+
+
+def check_attention_masked_bruteforce(o):
+    """With k*B_k < N, attention equals dense attention under the selection mask (brute force)."""
+    N, H_q, H_kv, d_h, d_idx, B_k, k = 160, 4, 2, 16, 8, 16, 3
+    inp = _attn_inputs(N, H_q, H_kv, d_h, d_idx, 5)
+    rows = np.arange(N)
+    sel, out, lse = o.prefill_rows(inp, rows, B_k, k)
+    sel_r = np.ascontiguousarray(sel.transpose(1, 0, 2))
+    assert np.array_equal(sel_r, ref.dense_selection(inp["q_idx"], inp["k_idx"], B_k, k))
+    want, want_lse = ref.masked_attention(inp["q"], inp["k"], inp["v"], ref.selection_mask(sel_r, N, B_k))
+    assert np.max(np.abs(out - want)) < 1e-12
+    assert np.max(np.abs(lse - want_lse)) < 1e-12
+
+
+def check_attention_zero_keys(o):
+    """k == 0: all logits equal, so out is the plain mean of v over the attended tokens, lse = log|T|."""
+    N, H_q, H_kv, d_h, d_idx, B_k, k = 90, 4, 2, 8, 8, 8, 3
+    inp = _attn_inputs(N, H_q, H_kv, d_h, d_idx, 9)
+    inp["k"] = np.zeros_like(inp["k"])
+    rows = np.arange(N)
+    sel, out, lse = o.prefill_rows(inp, rows, B_k, k)
+    V = bf16_bits_to_f64(inp["v"])
+    G = H_q // H_kv
+    for t, i in enumerate(rows):
+        for h in range(H_q):
+            r = h // G
+            toks = [j for b in sel[t, r] if b >= 0 for j in range(b * B_k, min((b + 1) * B_k, i + 1))]
+            assert np.max(np.abs(out[t, h] - V[toks, r].mean(axis=0))) < 1e-12
+            assert abs(lse[t, h] - math.log(len(toks))) < 1e-12
+
+
+def check_attention_k1_block_local(o):
+    """k = 1 keeps only the local block: causal attention inside each query's own block."""
+    N, H_q, H_kv, d_h, d_idx, B_k = 70, 2, 1, 8, 8, 16
+    inp = _attn_inputs(N, H_q, H_kv, d_h, d_idx, 13)
+    rows = np.arange(N)
+    sel, out, lse = o.prefill_rows(inp, rows, B_k, 1)
+    blk = np.arange(N) // B_k
+    allowed = (blk[:, None] == blk[None, :]) & np.tril(np.ones((N, N), dtype=bool))
+    want, want_lse = ref.masked_attention(inp["q"], inp["k"], inp["v"], allowed[None])
+    assert np.max(np.abs(out - want)) < 1e-12
+    assert np.max(np.abs(lse - want_lse)) < 1e-12
+
+
+def check_attention_hand_example(o):
+    """Three tokens, d_h = 4 (scale 1/2), q = (2,0,0,0), k_j = (j,0,0,0): logits 0, 1, 2 at row 2.
+
+    With v_j = (1, j, j^2, 0) the exact answer is (1, (e+2e^2)/Z, (e+4e^2)/Z, 0), Z = 1+e+e^2,
+    lse = log Z (B_k = 2, k = 2: row 2 keeps block 0 and its local block 1)."""
+    f = lambda a: f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+    inp = {
+        "q": f([[[2, 0, 0, 0]]] * 3),
+        "k": f([[[0, 0, 0, 0]], [[1, 0, 0, 0]], [[2, 0, 0, 0]]]),
+        "v": f([[[1, 0, 0, 0]], [[1, 1, 1, 0]], [[1, 2, 4, 0]]]),
+        "q_idx": f(np.zeros((3, 1, 1))),
+        "k_idx": f(np.zeros((3, 1, 1))),
+    }
+    sel, out, lse = o.prefill_rows(inp, np.array([0, 1, 2]), 2, 2)
+    e = math.e
+    Z = 1 + e + e * e
+    assert list(sel[2, 0]) == [0, 1]
+    want = np.array([1.0, (e + 2 * e * e) / Z, (e + 4 * e * e) / Z, 0.0])
+    assert np.max(np.abs(out[2, 0] - want)) < 1e-14, out[2, 0]
+    assert abs(lse[2, 0] - math.log(Z)) < 1e-14
+    # row 1 attends tokens 0 and 1 (logits 0 and 1); row 0 only token 0
+    Z1 = 1 + e
+    assert np.max(np.abs(out[1, 0] - np.array([1.0, e / Z1, e / Z1, 0.0]))) < 1e-14
+    assert np.max(np.abs(out[0, 0] - np.array([1.0, 0.0, 0.0, 0.0]))) < 1e-14
+    assert abs(lse[0, 0]) < 1e-14
+
+
+def check_combine_identity(o):
+    """Per-block softmax partials merged through their log-sum-exp equal the one-pass result."""
+    N, H_q, H_kv, d_h, d_idx, B_k, k = 200, 4, 2, 16, 8, 16, 4
+    inp = _attn_inputs(N, H_q, H_kv, d_h, d_idx, 21)
+    rows = np.array([0, 15, 16, 77, 130, 199])
+    sel, out, lse = o.prefill_rows(inp, rows, B_k, k)
+    Q, K, V = (bf16_bits_to_f64(inp[x]) for x in ("q", "k", "v"))
+    G = H_q // H_kv
+    for t, i in enumerate(rows):
+        for h in range(H_q):
+            r = h // G
+            parts = []
+            for b in sel[t, r]:
+                if b < 0:
+                    continue
+                js = np.arange(b * B_k, min((b + 1) * B_k, i + 1))
+                s = K[js, r] @ Q[i, h] / math.sqrt(d_h)
+                m = s.max()
+                w = np.exp(s - m)
+                parts.append((m + math.log(w.sum()), (w / w.sum()) @ V[js, r]))
+            L = np.logaddexp.reduce([p[0] for p in parts])
+            merged = sum(math.exp(p[0] - L) * p[1] for p in parts)
+            assert abs(L - lse[t, h]) < 1e-12
+            assert np.max(np.abs(merged - out[t, h])) < 1e-12
+
+
+def check_kv2q_bruteforce(o):
+    """The inversion lists equal a per-block brute-force scan, for oracle selections."""
+    N, H_kv, d_idx, B_k, k = 333, 2, 8, 16, 5
+    qi, ki = _idx_inputs(N, H_kv, d_idx, 31)
+    sel = o.select_all(qi, ki, B_k, k)
+    off, ent = o.kv2q(sel, B_k)
+    want = ref.brute_kv2q(sel, B_k)
+    nb = (N + B_k - 1) // B_k
+    for r in range(H_kv):
+        for b in range(nb):
+            assert np.array_equal(ent[r][off[r, b]:off[r, b + 1]], want[r][b]), (r, b)
+        assert off[r, -1] == sum(min(k, i // B_k + 1) for i in range(N))
+
+
+def check_decode_matches_prefill_row(o):
+    """Decode of a sequence of length L equals prefill row L-1 of the same data."""
+    B, L_max, H_q, H_kv, d_h, d_idx, B_k, k = 3, 150, 4, 2, 8, 8, 16, 3
+    lens = np.array([1, 77, 150], dtype=np.int32)
+    kc = normal_bf16((B, L_max, H_kv, d_h), 3, "dk")
+    vc = normal_bf16((B, L_max, H_kv, d_h), 3, "dv")
+    kic = int_uniform_bf16((B, L_max, H_kv, d_idx), -3, 3, 3, "dki")
+    q = normal_bf16((B, H_q, d_h), 3, "dq")
+    qi = int_uniform_bf16((B, H_kv, d_idx), -3, 3, 3, "dqi")
+    dec = {"q": q, "q_idx": qi, "k_cache": kc, "v_cache": vc, "k_idx_cache": kic, "lens": lens}
+    sel, out, lse = o.decode(dec, B_k, k)
+    for beta in range(B):
+        L = int(lens[beta])
+        inp = {"k": kc[beta, :L], "v": vc[beta, :L], "k_idx": kic[beta, :L],
+               "q": np.repeat(q[beta][None], L, 0), "q_idx": np.repeat(qi[beta][None], L, 0)}
+        s2, o2, l2 = o.prefill_rows(inp, np.array([L - 1]), B_k, k)
+        assert np.array_equal(sel[beta], s2[0])
+        assert np.max(np.abs(out[beta] - o2[0])) < 1e-13
+        assert np.max(np.abs(lse[beta] - l2[0])) < 1e-13
+
+
+ALL_CHECKS = [
+    check_selection_bruteforce,
+    check_selection_ties_closed_form,
+    check_selection_planted_winners,
+    check_selection_invariants,
+    check_attention_dense_invariant,
+    check_attention_masked_bruteforce,
+    check_attention_zero_keys,
+    check_attention_k1_block_local,
+    check_attention_hand_example,
+    check_combine_identity,
+    check_kv2q_bruteforce,
+    check_decode_matches_prefill_row,
+]
