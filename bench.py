@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MSA forward hot path (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one batch of synthetic input: the 128K-token planted
+prefill (index Top-k -> KV->Q inversion -> KV-outer attention -> LSE combine) followed by one decode
+step of 64 sequences against 16K-128K token caches. `value` is prefill tokens/s over all ranks
+(each rank processes its own independent sequence: weak scaling, no collective on the data path);
+decode tokens/s and every kernel's roofline fraction are reported alongside.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {msa,reference}]
+
+--impl reference times the plain CPU oracle (the reference arm of this build) on the host cores,
+on a bounded sample of the same workload, and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_long_idx_b200 import roofline, synth  # noqa: E402
+
+METRIC = "MSA prefill tokens/s @N=128K (64q/4kv heads), decode tok/s; % of roofline"
+UNIT = "tokens/s"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["msa", "reference"], default="msa")
+    ap.add_argument("--workload", default=synth.P128K.name, choices=sorted(synth.PREFILL_CONFIGS))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-oracle sample time")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------------ CPU oracle
+def oracle_rate(prefill_inputs, cfg, target_s: float):
+    """Oracle rows/s on a bounded sample of the workload's rows (selection + attention, all heads)."""
+    import oracle
+
+    o = oracle.default()
+
+    def run(n, seed):
+        rows = synth.sample_rows(cfg.N, cfg.B_k, n, seed)
+        t0 = time.perf_counter()
+        o.prefill_rows(prefill_inputs, rows, cfg.B_k, cfg.k)
+        return len(rows), time.perf_counter() - t0
+
+    n0, t0 = run(8, 101)
+    n = max(8, int(n0 * target_s / max(t0, 1e-3)))
+    n1, t1 = run(n, 202)
+    return {"value": n1 / t1, "unit": UNIT, "cores": o.max_threads(), "kind": "oracle",
+            "sample": f"{n1} uniformly sampled query rows (plus rows 0, B_k-1, B_k, N-1) of {cfg.name}: "
+                      f"index selection + exact sparse attention for all {cfg.H_q} heads, fp64, "
+                      f"{t1:.1f} s; value = rows/s"}
+
+
+def reference_arm(args, rank):
+    if rank != 0:
+        return
+    cfg = synth.PREFILL_CONFIGS[args.workload]
+    inputs = synth.prefill_inputs(cfg)
+    import oracle
+
+    o = oracle.default()
+    per_step = max(args.cpu_seconds / max(args.steps, 1), 2.0)
+    times, rows_done = [], []
+    for s in range(args.warmup + args.steps):
+        rows = synth.sample_rows(cfg.N, cfg.B_k, max(4, int(4 * per_step)), 1000 + s)
+        t0 = time.perf_counter()
+        o.prefill_rows(inputs, rows, cfg.B_k, cfg.k)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            rows_done.append(len(rows))
+    value = sum(rows_done) / sum(times)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(cfg, None),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": o.max_threads(), "kind": "oracle",
+                             "sample": f"per step {rows_done[0]} sampled query rows of {cfg.name} "
+                                       "(selection + attention, all heads)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------ GPU arm
+def workload_config(cfg, dcfg):
+    c = {"workload": cfg.name + (f" + {dcfg.name}" if dcfg else ""), "N": cfg.N, "H_q": cfg.H_q, "H_kv": cfg.H_kv,
+         "d_h": cfg.d_h, "d_idx": cfg.d_idx, "B_k": cfg.B_k, "k": cfg.k, "planted": cfg.planted,
+         "l2": "flushed before every timed step (512 MB write)"}
+    if dcfg:
+        c["decode"] = {"B": dcfg.B, "L_max": dcfg.L_max, "lens": f"uniform [{dcfg.len_lo}, {dcfg.len_hi}]"}
+    return c
+
+
+class ClockSampler:
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_arm(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_long_idx_b200 as msa
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    cfg = synth.PREFILL_CONFIGS[args.workload]
+    cfg = cfg.with_(seed=cfg.seed + 1000 * rank)  # independent sequence per rank
+    dcfg = None if args.no_decode else synth.DECODE64.with_(seed=synth.DECODE64.seed + 1000 * rank)
+
+    host = synth.prefill_inputs(cfg)
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = oracle_rate(host, cfg, args.cpu_seconds)  # before any GPU work
+
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+
+    t = {n: to_dev(a) for n, a in host.items()}
+    N, H_q, H_kv, d_h, d_idx, k = cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.k
+    block_idx = torch.empty((H_kv, N, k), dtype=torch.int32, device=dev)
+    L = msa.msa_kv2q_layout_get(N, H_kv, cfg.B_k, k)
+    kv = msa.KV2Q(L, torch.empty(L.total_bytes, dtype=torch.uint8, device=dev))
+    ws_kv = torch.empty(msa.api.lib.msa_build_kv2q_workspace_size(msa.api.ctypes.byref(L)), dtype=torch.uint8,
+                        device=dev)
+    ws_pf = torch.empty(msa.msa_sparse_prefill_workspace_size(N, H_q, H_kv, d_h, cfg.B_k, k), dtype=torch.uint8,
+                        device=dev)
+    out = torch.empty_like(t["q"])
+    lse = torch.empty((N, H_q), dtype=torch.float32, device=dev)
+    ws_idx = torch.empty(256, dtype=torch.uint8, device=dev)
+
+    if dcfg:
+        dh = synth.decode_inputs(dcfg)
+        dt = {n: to_dev(a) for n, a in dh.items()}
+        dout = torch.empty_like(dt["q"])
+        dlse = torch.empty((dcfg.B, dcfg.H_q), dtype=torch.float32, device=dev)
+        dbi = torch.empty((dcfg.B, dcfg.H_kv, dcfg.k), dtype=torch.int32, device=dev)
+        ws_dec = torch.empty(msa.api.lib.msa_sparse_decode_workspace_size(
+            dcfg.B, dcfg.L_max, dcfg.H_q, dcfg.H_kv, dcfg.d_h, dcfg.d_idx, dcfg.B_k, dcfg.k), dtype=torch.uint8,
+            device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        msa.msa_index_topk(t["q_idx"], t["k_idx"], cfg.B_k, k, block_idx=block_idx, workspace=ws_idx)
+        msa.api._check("msa_build_kv2q", msa.api.lib.msa_build_kv2q(
+            block_idx.data_ptr(), msa.api.ctypes.byref(L), kv.buf.data_ptr(), ws_kv.data_ptr(), ws_kv.numel(),
+            stream.cuda_stream))
+        msa.msa_sparse_prefill(t["q"], t["k"], t["v"], block_idx, kv, out=out, lse=lse, workspace=ws_pf)
+
+    def decode():
+        msa.msa_sparse_decode(dt["q"], dt["q_idx"], dt["k_cache"], dt["v_cache"], dt["k_idx_cache"], dt["lens"],
+                              dcfg.B_k, dcfg.k, out=dout, lse=dlse, block_idx_out=dbi, workspace=ws_dec)
+
+    for _ in range(args.warmup):
+        prefill()
+        if dcfg:
+            decode()
+    torch.cuda.synchronize()
+    for ws in (ws_idx, ws_kv, ws_pf) + ((ws_dec,) if dcfg else ()):
+        st = msa.msa_get_device_error(ws)
+        if st != 0:
+            raise RuntimeError(f"device error {msa.status_string(st)} during warm-up")
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    trace = msa.KernelTrace(64 * args.steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = msa.msa_launch_count()
+    with ClockSampler(uuid) as clocks:
+        wall0 = time.perf_counter()
+        with trace:
+            for s in range(args.steps):
+                flush.zero_()  # evict L2 between steps (outside the timed events)
+                ev[s][0].record()
+                prefill()
+                ev[s][1].record()
+                if dcfg:
+                    decode()
+                ev[s][2].record()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    launches = msa.msa_launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    pf_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    kern = trace.durations()
+
+    # max over ranks
+    tt = torch.tensor([sum(pf_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    pf_total, dec_total = tt.tolist()
+
+    # end-to-end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = {n: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory()
+               for n, a in host.items()}
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(p.numel() * p.element_size() for p in pin.values())
+        d2h = out_h.numel() * out_h.element_size()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        for s in range(args.e2e_steps):
+            flush.zero_()
+            e0.record()
+            for n in t:
+                t[n].copy_(pin[n], non_blocking=True)
+            prefill()
+            out_h.copy_(out, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        te = torch.tensor([tot], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * N * args.e2e_steps / (te.item() / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "note": "prefill through the public API: pinned host inputs copied in, out copied back"}
+
+    if rank != 0:
+        return
+    value = world * N * args.steps / (pf_total / 1000.0)
+    kstats = {}
+    fl_main = roofline.main_branch_flops(N, H_q, d_h, k, cfg.B_k)
+    fl_idx = roofline.index_branch_flops(N, H_kv, d_idx)
+    algo = {"index_topk": ("tensor", fl_idx), "attn": ("tensor", fl_main),
+            "combine": ("hbm", roofline.combine_bytes(N, H_q, H_kv, d_h, k, cfg.B_k))}
+    if dcfg:
+        db = roofline.decode_bytes(dh["lens"], dcfg.H_q, dcfg.H_kv, dcfg.d_h, dcfg.d_idx, dcfg.k, dcfg.B_k)
+        algo["dec_pool"] = ("hbm", db["dec_pool"])
+        algo["dec_attn"] = ("hbm", db["dec_attn"])
+    for name, durs in kern.items():
+        per_step = sum(durs) / args.steps
+        ent = {"ms_per_step": per_step, "launches_per_step": len(durs) / args.steps}
+        if name in algo:
+            bound, work = algo[name]
+            if bound == "tensor":
+                ach = work / (per_step / 1000.0) / 1e12
+                ent.update({"bound": "tensor", "achieved": ach, "unit": "TFLOP/s", "peak": peaks["bf16_tflops"],
+                            "frac": ach / peaks["bf16_tflops"], "algorithmic": work})
+            else:
+                ach = work / (per_step / 1000.0) / 1e9
+                ent.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                            "frac": ach / peaks["hbm_gbs"], "algorithmic": work})
+        kstats[name] = ent
+    # dominant kernel of the prefill step
+    dom = max((n for n in ("index_topk", "attn", "combine") if n in kstats), key=lambda n: kstats[n]["ms_per_step"])
+    d = kstats[dom]
+    roof = {"kernel": dom, "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
+            "frac": d["frac"], "traffic": None, "peak_source": peaks["source"] + " (burst)"}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": (pf_total + dec_total) / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(cfg, dcfg), parallelism=f"replicas x{world} (independent sequences)"),
+            "prefill_ms_per_step": pf_total / args.steps,
+            "decode": ({"value": world * dcfg.B * args.steps / (dec_total / 1000.0), "unit": UNIT,
+                        "ms_per_step": dec_total / args.steps} if dcfg else None),
+            "roofline": roof, "kernels": kstats, "cpu_baseline": cpu_base, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clocks.summary(), "wall_s_timed": wall}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        gpu_arm(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

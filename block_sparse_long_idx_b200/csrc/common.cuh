@@ -1,0 +1,120 @@
+// common.cuh -- shared definitions of the MSA CUDA library (device error word, limits, launchers).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "msa.h"
+
+namespace msa {
+
+// Every bounded wait gives up after this many SM clock cycles (~1 s at 2 GHz) and records
+// MSA_ERR_TIMEOUT in the device error word.
+constexpr long long kWaitLimit = 2000000000LL;
+
+constexpr int kBk = 128;       // KV block size this build supports (one tensor-core tile)
+constexpr int kMaxK = 16;      // largest k
+constexpr int kMaxN = 1 << 21; // largest sequence length (nb <= 16384)
+
+// Device error word: the first 16 bytes of every workspace. [0] = status code, [1] = detail.
+struct ErrWord {
+    int code;
+    int detail;
+    int pad[2];
+};
+
+__device__ __forceinline__ void report_error(int* word, int code, int detail)
+{
+    if (atomicCAS(word, 0, code) == 0) word[1] = detail;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Opt-in per-kernel event tracing and the launch counter (msa_trace_set / msa_launch_count).
+void trace_begin(cudaStream_t s);
+void trace_end(cudaStream_t s, int kernel_id);
+void note_launch(int n);
+
+// ---------------------------------------------------------------------------------------------
+// launchers implemented in the .cu files
+// ---------------------------------------------------------------------------------------------
+struct IndexTopkArgs {
+    const uint16_t* q_idx;
+    const uint16_t* k_idx;
+    int64_t N;
+    int H_kv, d_idx, k;
+    int32_t* block_idx;
+    int* err;
+};
+cudaError_t launch_index_topk(const IndexTopkArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                              cudaStream_t s);
+
+struct Kv2qArgs {
+    const int32_t* block_idx;
+    int64_t N;
+    int H_kv, k, nb, window, chunk, n_windows;
+    int32_t* offsets;
+    int32_t* entries;
+    msa_work_item* items;
+    int32_t* window_items;
+    int32_t* counts; // [H_kv][nb][n_windows]
+    int32_t* bases;  // [H_kv][nb][n_windows]
+    int64_t max_items;
+    int32_t* scan_tmp;
+    int* err;
+};
+cudaError_t launch_kv2q(const Kv2qArgs& a, cudaStream_t s);
+size_t kv2q_scan_tmp_bytes(int64_t n, int H_kv);
+
+struct AttnArgs {
+    int64_t N;
+    int H_q, H_kv, d_h, k;
+    const int32_t* entries;     // [H_kv][N*k]
+    const msa_work_item* items; // work list
+    const int32_t* window_items;
+    int w0, w1;                 // windows of this pass
+    int64_t row0;               // first row of the pass (= w0 * window)
+    int64_t rows_pass;          // rows the partial buffers hold
+    uint16_t* o_part;           // [rows][k][H_q][d_h]
+    float* lse_part;            // [rows][k][H_q]
+    int* err;
+};
+cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                               const CUtensorMap& vmap, cudaStream_t s);
+
+struct CombineArgs {
+    int64_t row0, n_rows; // rows [row0, row0+n_rows) of the sequence
+    int H_q, d_h, k;
+    int64_t local_of_row_div; // B_k: n_sel(i) = min(k, i / B_k + 1)
+    const uint16_t* o_part;   // [n_rows][k][H_q][d_h]
+    const float* lse_part;    // [n_rows][k][H_q]
+    const int32_t* nsel;      // optional per-row count of valid slots (decode), else NULL
+    uint16_t* out;            // [*, H_q, d_h] rows offset by row0
+    float* lse;               // nullable
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+struct DecodeArgs {
+    const uint16_t* q;
+    const uint16_t* q_idx;
+    const uint16_t* k_cache;
+    const uint16_t* v_cache;
+    const uint16_t* k_idx_cache;
+    const int32_t* lens;
+    int B;
+    int64_t L_max;
+    int H_q, H_kv, d_h, d_idx, k;
+    float* pooled;        // [B][H_kv][nb_max]
+    int32_t* sel;         // [B][H_kv][k]
+    int32_t* nsel;        // [B]
+    uint16_t* o_part;     // [B][k][H_q][d_h]
+    float* lse_part;      // [B][k][H_q]
+    uint16_t* out;
+    float* lse;
+    int32_t* block_idx_out;
+    int* err;
+};
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+} // namespace msa

@@ -1,0 +1,458 @@
+// msa_api.cu -- the C ABI of libmsa_b200.so (declared in include/msa.h): host-side validation,
+// workspace carving, TMA descriptor encoding and kernel launches. No allocation, no host sync.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+using namespace msa;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 tensor [n2][n1][n0] (row-major), box {b0, b1, b2}.
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t b0, uint32_t b1,
+                 uint32_t b2, CUtensorMapSwizzle sw)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {n0, n1, n2};
+    const cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+    const cuuint32_t box[3] = {b0, b1, b2};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+bool injected(const char* name)
+{
+    const char* v = getenv("MSA_FAULT_INJECT");
+    return v && strcmp(v, name) == 0;
+}
+
+constexpr size_t kErrBytes = 256;
+constexpr int kDefaultWindow = 2048;
+constexpr int kDefaultChunk = 512;
+
+size_t kv2q_internal_tmp(const msa_kv2q_layout& L)
+{
+    return kv2q_scan_tmp_bytes((int64_t)L.H_kv * L.nb * L.n_windows, L.H_kv);
+}
+
+thread_local char g_last_error[256] = "no error";
+
+// Records the failing CUDA call of the last MSA_ERR_CUDA (per thread) for msa_last_error_string().
+msa_status cuda_status(cudaError_t e, const char* site)
+{
+    if (e == cudaSuccess) return MSA_OK;
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", site, cudaGetErrorName(e), cudaGetErrorString(e));
+    return MSA_ERR_CUDA;
+}
+
+msa_trace* g_trace = nullptr;
+std::atomic<uint64_t> g_launches{0};
+
+} // namespace
+
+namespace msa {
+
+// A record that fails (e.g. a handle that is not a live event) ends tracing for this record and
+// clears the error, so that it is never mistaken for a launch failure.
+static bool trace_record(msa_trace* t, int slot, cudaStream_t s)
+{
+    if (t->events[slot] && cudaEventRecord((cudaEvent_t)t->events[slot], s) == cudaSuccess) return true;
+    cudaGetLastError();
+    t->capacity = t->count;
+    return false;
+}
+
+void trace_begin(cudaStream_t s)
+{
+    msa_trace* t = g_trace;
+    if (t && t->count + 2 <= t->capacity) trace_record(t, t->count, s);
+}
+
+void trace_end(cudaStream_t s, int kernel_id)
+{
+    msa_trace* t = g_trace;
+    if (t && t->count + 2 <= t->capacity && trace_record(t, t->count + 1, s)) {
+        t->kernel_ids[t->count / 2] = kernel_id;
+        t->count += 2;
+    }
+}
+
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+} // namespace msa
+
+extern "C" {
+
+void msa_trace_set(msa_trace* trace) { g_trace = trace; }
+
+const char* msa_last_error_string(void) { return g_last_error; }
+
+uint64_t msa_launch_count(void) { return g_launches.load(); }
+
+const char* msa_status_string(msa_status s)
+{
+    switch (s) {
+    case MSA_OK: return "MSA_OK";
+    case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG";
+    case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED";
+    case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE";
+    case MSA_ERR_CUDA: return "MSA_ERR_CUDA";
+    case MSA_ERR_TIMEOUT: return "MSA_ERR_TIMEOUT";
+    case MSA_ERR_DEVICE_CHECK: return "MSA_ERR_DEVICE_CHECK";
+    }
+    return "MSA_ERR_UNKNOWN";
+}
+
+msa_status msa_get_device_error(const void* workspace, msa_stream_t stream)
+{
+    if (!workspace) return MSA_ERR_INVALID_ARG;
+    int h[2] = {0, 0};
+    if (cudaMemcpyAsync(h, workspace, sizeof h, cudaMemcpyDeviceToHost, (cudaStream_t)stream) != cudaSuccess ||
+        cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+        return MSA_ERR_CUDA;
+    return (msa_status)h[0];
+}
+
+// ------------------------------------------------------------------------------------ index_topk
+size_t msa_index_topk_workspace_size(int64_t, int, int, int, int) { return kErrBytes; }
+
+msa_status msa_index_topk(const msa_bf16* q_idx, const msa_bf16* k_idx, int64_t N, int H_kv, int d_idx, int B_k,
+                          int k, int32_t* block_idx, void* workspace, size_t workspace_bytes, msa_stream_t stream)
+{
+    if (!q_idx || !k_idx || !block_idx || !workspace || N < 1 || H_kv < 1 || k < 1 || d_idx < 1 || B_k < 1)
+        return MSA_ERR_INVALID_ARG;
+    if (!aligned(q_idx, 16) || !aligned(k_idx, 16) || !aligned(block_idx, 4) || !aligned(workspace, 256))
+        return MSA_ERR_INVALID_ARG;
+    if (B_k != kBk || k > kMaxK || !(d_idx == 32 || d_idx == 64 || d_idx == 128) || N > kMaxN || H_kv > 65535)
+        return MSA_ERR_UNSUPPORTED;
+    if (workspace_bytes < kErrBytes) return MSA_ERR_WORKSPACE;
+    if (injected("msa_index_topk")) return MSA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    CUtensorMap qmap, kmap;
+    const uint32_t box0 = d_idx < 64 ? (uint32_t)d_idx : 64u;
+    const CUtensorMapSwizzle sw = d_idx == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_map_3d(&qmap, q_idx, d_idx, H_kv, N, box0, 1, kBk, sw) ||
+        !make_map_3d(&kmap, k_idx, d_idx, H_kv, N, box0, 1, kBk, sw))
+        return MSA_ERR_INVALID_ARG;
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    IndexTopkArgs a{q_idx, k_idx, N, H_kv, d_idx, k, block_idx, (int*)workspace};
+    trace_begin(s);
+    const cudaError_t e = launch_index_topk(a, qmap, kmap, s);
+    trace_end(s, MSA_KERNEL_INDEX_TOPK);
+    return cuda_status(e, "index_topk launch");
+}
+
+// ------------------------------------------------------------------------------------ kv2q
+msa_status msa_kv2q_layout_get(int64_t N, int H_kv, int B_k, int k, int window, int chunk, msa_kv2q_layout* L)
+{
+    if (!L || N < 1 || H_kv < 1 || B_k < 1 || k < 1 || window < 0 || chunk < 0) return MSA_ERR_INVALID_ARG;
+    if (B_k != kBk || k > kMaxK || N > kMaxN) return MSA_ERR_UNSUPPORTED;
+    if (window == 0) window = kDefaultWindow;
+    if (chunk == 0) chunk = kDefaultChunk < window ? kDefaultChunk : window;
+    if (window % kBk != 0 || chunk > window) return MSA_ERR_INVALID_ARG;
+    memset(L, 0, sizeof *L);
+    L->N = N;
+    L->H_kv = H_kv;
+    L->B_k = B_k;
+    L->k = k;
+    L->nb = (int32_t)((N + B_k - 1) / B_k);
+    L->window = window;
+    L->chunk = chunk;
+    L->n_windows = (int32_t)((N + window - 1) / window);
+    int64_t max_items = 0;
+    for (int64_t w = 0; w < L->n_windows; ++w) {
+        const int64_t lo = w * window, hi = (w + 1) * window < N ? (w + 1) * window : N;
+        const int64_t vis = (hi - 1) / B_k + 1;
+        max_items += (int64_t)H_kv * (vis + ((hi - lo) * k + chunk - 1) / chunk);
+    }
+    L->max_items = max_items;
+    const int64_t n = (int64_t)H_kv * L->nb * L->n_windows;
+    size_t off = 0;
+    L->offsets = off;
+    off = align_up(off + (size_t)H_kv * (L->nb + 1) * 4, 256);
+    L->entries = off;
+    off = align_up(off + (size_t)H_kv * N * k * 4, 256);
+    L->items = off;
+    off = align_up(off + (size_t)max_items * sizeof(msa_work_item), 256);
+    L->window_items = off;
+    off = align_up(off + (size_t)(L->n_windows + 1) * 4, 256);
+    L->counts = off;
+    off = align_up(off + (size_t)2 * n * 4, 256);
+    L->bases = off;
+    off = align_up(off + (size_t)n * 4, 256);
+    L->total_bytes = off;
+    return MSA_OK;
+}
+
+size_t msa_build_kv2q_workspace_size(const msa_kv2q_layout* L)
+{
+    return L ? kErrBytes + kv2q_internal_tmp(*L) : 0;
+}
+
+static msa_status build_kv2q_impl(const int32_t* block_idx, const msa_kv2q_layout* L, void* kv2q, int* err,
+                                  void* tmp, cudaStream_t s)
+{
+    uint8_t* base = (uint8_t*)kv2q;
+    Kv2qArgs a;
+    a.block_idx = block_idx;
+    a.N = L->N;
+    a.H_kv = L->H_kv;
+    a.k = L->k;
+    a.nb = L->nb;
+    a.window = L->window;
+    a.chunk = L->chunk;
+    a.n_windows = L->n_windows;
+    a.offsets = (int32_t*)(base + L->offsets);
+    a.entries = (int32_t*)(base + L->entries);
+    a.items = (msa_work_item*)(base + L->items);
+    a.window_items = (int32_t*)(base + L->window_items);
+    a.counts = (int32_t*)(base + L->counts);
+    a.bases = (int32_t*)(base + L->bases);
+    a.max_items = L->max_items;
+    a.scan_tmp = (int32_t*)tmp;
+    a.err = err;
+    trace_begin(s);
+    const cudaError_t e = launch_kv2q(a, s);
+    trace_end(s, MSA_KERNEL_KV2Q);
+    return cuda_status(e, "kv2q launch");
+}
+
+static bool layout_ok(const msa_kv2q_layout* L)
+{
+    msa_kv2q_layout ref;
+    if (msa_kv2q_layout_get(L->N, L->H_kv, L->B_k, L->k, L->window, L->chunk, &ref) != MSA_OK) return false;
+    return ref.nb == L->nb && ref.n_windows == L->n_windows && ref.max_items == L->max_items &&
+           ref.offsets == L->offsets && ref.entries == L->entries && ref.items == L->items &&
+           ref.window_items == L->window_items && ref.counts == L->counts && ref.bases == L->bases &&
+           ref.total_bytes == L->total_bytes;
+}
+
+msa_status msa_build_kv2q(const int32_t* block_idx, const msa_kv2q_layout* L, void* kv2q, void* workspace,
+                          size_t workspace_bytes, msa_stream_t stream)
+{
+    if (!block_idx || !L || !kv2q || !workspace) return MSA_ERR_INVALID_ARG;
+    if (!layout_ok(L) || !aligned(kv2q, 256) || !aligned(workspace, 256) || !aligned(block_idx, 4))
+        return MSA_ERR_INVALID_ARG;
+    if (workspace_bytes < msa_build_kv2q_workspace_size(L)) return MSA_ERR_WORKSPACE;
+    if (injected("msa_build_kv2q")) return MSA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    return build_kv2q_impl(block_idx, L, kv2q, (int*)workspace, (uint8_t*)workspace + kErrBytes, s);
+}
+
+// ------------------------------------------------------------------------------------ sparse prefill
+static size_t partial_row_bytes(int H_q, int d_h, int k) { return (size_t)k * H_q * ((size_t)d_h * 2 + 4); }
+
+size_t msa_sparse_prefill_workspace_size(int64_t N, int H_q, int H_kv, int d_h, int B_k, int k,
+                                         int64_t max_rows_per_pass, int internal_kv2q)
+{
+    msa_kv2q_layout L;
+    if (msa_kv2q_layout_get(N, H_kv, B_k, k, 0, 0, &L) != MSA_OK || H_q < 1) return 0;
+    int64_t rows = max_rows_per_pass <= 0 || max_rows_per_pass > N ? N : max_rows_per_pass;
+    rows = (rows + L.window - 1) / L.window * L.window;
+    size_t sz = kErrBytes + 512; // error word + alignment slack of the partial buffers
+    if (internal_kv2q) sz += align_up(L.total_bytes, 256) + align_up(kv2q_internal_tmp(L), 256);
+    sz += align_up((size_t)rows * k * H_q * d_h * 2, 256) + align_up((size_t)rows * k * H_q * 4, 256);
+    return sz;
+}
+
+msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_bf16* v, int64_t N, int H_q, int H_kv,
+                              int d_h, int B_k, int k, const int32_t* block_idx, const msa_kv2q_layout* layout,
+                              const void* kv2q, msa_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
+                              msa_stream_t stream)
+{
+    if (!q || !kk || !v || !block_idx || !out || !workspace || N < 1 || H_q < 1 || H_kv < 1 || d_h < 1 || k < 1)
+        return MSA_ERR_INVALID_ARG;
+    if ((layout == nullptr) != (kv2q == nullptr)) return MSA_ERR_INVALID_ARG;
+    if (H_q % H_kv != 0) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(kk, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
+        (lse && !aligned(lse, 4)))
+        return MSA_ERR_INVALID_ARG;
+    const int G = H_q / H_kv;
+    if (B_k != kBk || k > kMaxK || !(d_h == 64 || d_h == 128) || !pow2(G) || G > 128 || N > kMaxN)
+        return MSA_ERR_UNSUPPORTED;
+    if (layout && (!layout_ok(layout) || layout->N != N || layout->H_kv != H_kv || layout->k != k))
+        return MSA_ERR_INVALID_ARG;
+    if (injected("msa_sparse_prefill")) return MSA_ERR_CUDA;
+
+    msa_kv2q_layout Lint;
+    const msa_kv2q_layout* L = layout;
+    uint8_t* ws = (uint8_t*)workspace;
+    size_t used = kErrBytes;
+    const void* kv = kv2q;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    if (!L) {
+        msa_kv2q_layout_get(N, H_kv, B_k, k, 0, 0, &Lint);
+        L = &Lint;
+        const size_t need = align_up(L->total_bytes, 256) + align_up(kv2q_internal_tmp(*L), 256);
+        if (workspace_bytes < used + need) return MSA_ERR_WORKSPACE;
+        void* kvbuf = ws + used;
+        void* tmp = ws + used + align_up(L->total_bytes, 256);
+        used += need;
+        msa_status st = build_kv2q_impl(block_idx, L, kvbuf, (int*)workspace, tmp, s);
+        if (st != MSA_OK) return st;
+        kv = kvbuf;
+    }
+    // rows of partials the remaining workspace holds, in whole windows
+    const size_t per_row = partial_row_bytes(H_q, d_h, k);
+    if (workspace_bytes <= used + 512) return MSA_ERR_WORKSPACE;
+    int64_t rows_cap = (int64_t)((workspace_bytes - used - 512) / per_row);
+    int64_t wins_per_pass = rows_cap / L->window;
+    if (wins_per_pass < 1) return MSA_ERR_WORKSPACE;
+    if (wins_per_pass > L->n_windows) wins_per_pass = L->n_windows;
+    const int64_t rows_pass = wins_per_pass * L->window;
+    uint16_t* o_part = (uint16_t*)(ws + used);
+    float* lse_part = (float*)(ws + used + align_up((size_t)rows_pass * k * H_q * d_h * 2, 256));
+
+    CUtensorMap qmap, kmap, vmap;
+    if (!make_map_3d(&qmap, q, d_h, H_q, N, 64, G, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d(&kmap, kk, d_h, H_kv, N, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d(&vmap, v, d_h, H_kv, N, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B))
+        return MSA_ERR_INVALID_ARG;
+
+    const uint8_t* kvb = (const uint8_t*)kv;
+    for (int64_t w0 = 0; w0 < L->n_windows; w0 += wins_per_pass) {
+        const int64_t w1 = w0 + wins_per_pass < L->n_windows ? w0 + wins_per_pass : L->n_windows;
+        AttnArgs a;
+        a.N = N;
+        a.H_q = H_q;
+        a.H_kv = H_kv;
+        a.d_h = d_h;
+        a.k = k;
+        a.entries = (const int32_t*)(kvb + L->entries);
+        a.items = (const msa_work_item*)(kvb + L->items);
+        a.window_items = (const int32_t*)(kvb + L->window_items);
+        a.w0 = (int)w0;
+        a.w1 = (int)w1;
+        a.row0 = w0 * L->window;
+        a.rows_pass = rows_pass;
+        a.o_part = o_part;
+        a.lse_part = lse_part;
+        a.err = (int*)workspace;
+        trace_begin(s);
+        const cudaError_t ea = launch_sparse_attn(a, qmap, kmap, vmap, s);
+        trace_end(s, MSA_KERNEL_ATTN);
+        if (ea != cudaSuccess) return cuda_status(ea, "attention launch");
+        CombineArgs c;
+        c.row0 = a.row0;
+        c.n_rows = (w1 * L->window < N ? w1 * L->window : N) - a.row0;
+        c.H_q = H_q;
+        c.d_h = d_h;
+        c.k = k;
+        c.local_of_row_div = kBk;
+        c.o_part = o_part;
+        c.lse_part = lse_part;
+        c.nsel = nullptr;
+        c.out = out;
+        c.lse = lse;
+        trace_begin(s);
+        const cudaError_t ec = launch_combine(c, s);
+        trace_end(s, MSA_KERNEL_COMBINE);
+        if (ec != cudaSuccess) return cuda_status(ec, "combine launch");
+    }
+    return MSA_OK;
+}
+
+// ------------------------------------------------------------------------------------ decode
+size_t msa_sparse_decode_workspace_size(int B, int64_t L_max, int H_q, int H_kv, int d_h, int, int B_k, int k)
+{
+    if (B < 1 || L_max < 1 || B_k < 1 || k < 1) return 0;
+    const int64_t nb_max = (L_max + B_k - 1) / B_k;
+    size_t sz = kErrBytes;
+    sz += align_up((size_t)B * H_kv * nb_max * 4, 256);
+    sz += align_up((size_t)B * H_kv * k * 4, 256);
+    sz += align_up((size_t)B * 4, 256);
+    sz += align_up((size_t)B * k * H_q * d_h * 2, 256);
+    sz += align_up((size_t)B * k * H_q * 4, 256);
+    return sz;
+}
+
+msa_status msa_sparse_decode(const msa_bf16* q, const msa_bf16* q_idx, const msa_bf16* k_cache,
+                             const msa_bf16* v_cache, const msa_bf16* k_idx_cache, const int32_t* lens, int B,
+                             int64_t L_max, int H_q, int H_kv, int d_h, int d_idx, int B_k, int k, msa_bf16* out,
+                             float* lse, int32_t* block_idx_out, void* workspace, size_t workspace_bytes,
+                             msa_stream_t stream)
+{
+    if (!q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !lens || !out || !workspace || B < 1 || L_max < 1 ||
+        H_q < 1 || H_kv < 1 || d_h < 1 || d_idx < 1 || k < 1)
+        return MSA_ERR_INVALID_ARG;
+    if (H_q % H_kv != 0) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(q_idx, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(k_idx_cache, 16) || !aligned(lens, 4) || !aligned(out, 16) || !aligned(workspace, 256) ||
+        (lse && !aligned(lse, 4)) || (block_idx_out && !aligned(block_idx_out, 4)))
+        return MSA_ERR_INVALID_ARG;
+    const int G = H_q / H_kv;
+    const int lanes_per_pos = H_kv * d_idx / 8;
+    if (B_k != kBk || k > kMaxK || !(d_h == 64 || d_h == 128) || !pow2(G) || G > 16 ||
+        !(d_idx == 32 || d_idx == 64 || d_idx == 128) || !pow2(lanes_per_pos) || lanes_per_pos > 32 ||
+        L_max > kMaxN || B > 65535 || H_kv > 65535)
+        return MSA_ERR_UNSUPPORTED;
+    if (workspace_bytes < msa_sparse_decode_workspace_size(B, L_max, H_q, H_kv, d_h, d_idx, B_k, k))
+        return MSA_ERR_WORKSPACE;
+    if (injected("msa_sparse_decode")) return MSA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* ws = (uint8_t*)workspace;
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    const int64_t nb_max = (L_max + B_k - 1) / B_k;
+    size_t off = kErrBytes;
+    DecodeArgs a;
+    a.q = q;
+    a.q_idx = q_idx;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.k_idx_cache = k_idx_cache;
+    a.lens = lens;
+    a.B = B;
+    a.L_max = L_max;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.d_h = d_h;
+    a.d_idx = d_idx;
+    a.k = k;
+    a.pooled = (float*)(ws + off);
+    off += align_up((size_t)B * H_kv * nb_max * 4, 256);
+    a.sel = (int32_t*)(ws + off);
+    off += align_up((size_t)B * H_kv * k * 4, 256);
+    a.nsel = (int32_t*)(ws + off);
+    off += align_up((size_t)B * 4, 256);
+    a.o_part = (uint16_t*)(ws + off);
+    off += align_up((size_t)B * k * H_q * d_h * 2, 256);
+    a.lse_part = (float*)(ws + off);
+    a.out = out;
+    a.lse = lse;
+    a.block_idx_out = block_idx_out;
+    a.err = (int*)workspace;
+    return cuda_status(launch_decode(a, s), "decode launch");
+}
+
+} // extern "C"

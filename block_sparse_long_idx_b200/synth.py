@@ -224,16 +224,26 @@ def decode_lens(cfg: DecodeConfig) -> np.ndarray:
     return _rng(cfg.seed, "lens", 0).integers(cfg.len_lo, cfg.len_hi + 1, size=cfg.B).astype(np.int32)
 
 
-def decode_inputs(cfg: DecodeConfig) -> dict:
-    """Caches [B, L_max, H_kv, d] (positions >= len are present but unused), one query per sequence."""
+def decode_inputs(cfg: DecodeConfig, lens=None) -> dict:
+    """Caches [B, L_max, H_kv, d] holding each sequence's first len tokens (the rest is zero and never
+    read), one query per sequence. Each sequence's cache rows come from their own streams."""
     B, L = cfg.B, cfg.L_max
+    lens = decode_lens(cfg) if lens is None else np.asarray(lens, dtype=np.int32)
+    kc = np.zeros((B, L, cfg.H_kv, cfg.d_h), dtype=np.uint16)
+    vc = np.zeros_like(kc)
+    kic = np.zeros((B, L, cfg.H_kv, cfg.d_idx), dtype=np.uint16)
+    for b in range(B):
+        n = int(min(max(lens[b], 0), L))
+        kc[b, :n] = normal_bf16((n, cfg.H_kv, cfg.d_h), cfg.seed, f"k_cache/{b}")
+        vc[b, :n] = normal_bf16((n, cfg.H_kv, cfg.d_h), cfg.seed, f"v_cache/{b}")
+        kic[b, :n] = int_uniform_bf16((n, cfg.H_kv, cfg.d_idx), -3, 3, cfg.seed, f"k_idx_cache/{b}")
     return {
-        "lens": decode_lens(cfg),
+        "lens": lens,
         "q": normal_bf16((B, cfg.H_q, cfg.d_h), cfg.seed, "dq"),
         "q_idx": int_uniform_bf16((B, cfg.H_kv, cfg.d_idx), -3, 3, cfg.seed, "dq_idx"),
-        "k_cache": normal_bf16((B, L, cfg.H_kv, cfg.d_h), cfg.seed, "k_cache"),
-        "v_cache": normal_bf16((B, L, cfg.H_kv, cfg.d_h), cfg.seed, "v_cache"),
-        "k_idx_cache": int_uniform_bf16((B, L, cfg.H_kv, cfg.d_idx), -3, 3, cfg.seed, "k_idx_cache"),
+        "k_cache": kc,
+        "v_cache": vc,
+        "k_idx_cache": kic,
     }
 
 

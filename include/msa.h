@@ -1,0 +1,231 @@
+/*
+ * msa.h -- C ABI of libmsa_b200.so, the B200 (sm_100a) forward hot path of MiniMax Sparse Attention.
+ *
+ * Sources for what each call computes:
+ *   [EXPL] "MiniMax Sparse Attention" explainer page: section 01 (causal GQA attention, G adjacent
+ *          query heads share one KV head), section 02 (two-stage Index / Attn decomposition),
+ *          Figure 1 (Index Branch: score, Block Max Pooling, Top-k per (query, GQA group) with the
+ *          forced local block), section 04 (fixed budget k*B_k = 16*128), section 05-1 (exp-free
+ *          Top-k), section 05-2 (KV-outer sparse attention, query concatenation, pre-scheduled
+ *          chunking, two-stage forward with an LSE split-K combine, LSE emitted for the backward).
+ *   [ABS]  The paper abstract ("MiniMax Sparse Attention", arXiv 2606.13392): Top-k per GQA
+ *          group, exact block-sparse attention over the selected blocks, prefill and decoding.
+ *
+ * Conventions shared by every entry point
+ *   - bf16 tensors are passed as uint16_t bit patterns (msa_bf16).
+ *   - Every tensor pointer is a DEVICE pointer into memory the caller allocated and owns; the
+ *     library never allocates, frees or retains memory and keeps no global state besides the
+ *     cached driver entry point used to encode TMA descriptors.
+ *   - All work is enqueued asynchronously on `stream`; nothing synchronises the host.
+ *   - Arguments are validated on the host before anything is enqueued; a rejected call enqueues
+ *     nothing and returns MSA_ERR_INVALID_ARG (bad pointer / shape / alignment),
+ *     MSA_ERR_UNSUPPORTED (a valid shape this build has no kernel for) or MSA_ERR_WORKSPACE
+ *     (workspace too small). Launch failures return MSA_ERR_CUDA.
+ *   - Conditions only the device can see (a bounded wait that expired, a decode length outside
+ *     [1, L_max]) are recorded in the device error word at the start of the workspace and read
+ *     with msa_get_device_error(). No kernel traps.
+ *   - Workspaces must be 256-byte aligned. Every entry point clears its own device error word.
+ *   - Inputs must be finite. No C++ exception crosses this boundary.
+ *
+ * Supported shapes in this build: B_k = 128; 1 <= k <= 16; d_idx in {32, 64, 128};
+ * d_h in {64, 128}; G = H_q / H_kv a power of two with G <= 128 (prefill) and G <= 16 (decode);
+ * 1 <= N <= 2^21.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+typedef uint16_t msa_bf16;
+typedef struct CUstream_st* msa_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1,
+    MSA_ERR_UNSUPPORTED = 2,
+    MSA_ERR_WORKSPACE = 3,
+    MSA_ERR_CUDA = 4,
+    MSA_ERR_TIMEOUT = 5,
+    MSA_ERR_DEVICE_CHECK = 6
+} msa_status;
+
+/* Human-readable name of a status code (static storage). */
+MSA_API const char* msa_status_string(msa_status status);
+
+/* The CUDA call behind the calling thread's most recent MSA_ERR_CUDA, with its error name. */
+MSA_API const char* msa_last_error_string(void);
+
+/*
+ * Reads the device error word of a workspace previously passed to an entry point (waits for
+ * `stream` to finish). Returns MSA_OK, MSA_ERR_TIMEOUT (a bounded wait inside a kernel expired)
+ * or MSA_ERR_DEVICE_CHECK (an input only the device can check was out of range), or
+ * MSA_ERR_CUDA if the read itself failed.
+ */
+MSA_API msa_status msa_get_device_error(const void* workspace, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Index Branch: fused index score + block max-pool + exp-free Top-k      [EXPL Fig. 1, 05-1]
+ *
+ * For every query row i and GQA group r:
+ *   s_j      = q_idx[i, r, :] . k_idx[j, r, :]            (fp32 accumulation of bf16 products)
+ *   S[i,r,b] = max over j in block b of s_j, for the fully visible blocks b < floor(i / B_k)
+ *   set      = the k-1 blocks with the largest S (equal scores: lower block first) plus the local
+ *              block floor(i / B_k); all visible blocks when floor(i / B_k) + 1 <= k.
+ * No exp is evaluated (softmax preserves order). The pooled N x N/B_k score matrix is never
+ * written to memory: scores go from tensor memory straight into per-row register Top-k lists.
+ *
+ *   q_idx, k_idx : [N, H_kv, d_idx] bf16, row-major, 16-byte aligned
+ *   block_idx    : [H_kv, N, k] int32 out; each row ascending, padded with -1
+ *   workspace    : >= msa_index_topk_workspace_size(...) bytes (error word + scheduler state)
+ * Index inputs whose scores are exact in fp32 (e.g. small integers) give selections identical
+ * to an exact-arithmetic reference.
+ * ------------------------------------------------------------------------------------------ */
+MSA_API size_t msa_index_topk_workspace_size(int64_t N, int H_kv, int d_idx, int B_k, int k);
+
+MSA_API msa_status msa_index_topk(const msa_bf16* q_idx, const msa_bf16* k_idx, int64_t N, int H_kv, int d_idx, int B_k,
+                          int k, int32_t* block_idx, void* workspace, size_t workspace_bytes, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * KV -> Q inversion with pre-scheduled chunking                                  [EXPL 05-2]
+ *
+ * Turns the per-query selections into per-KV-block lists of the query rows that selected the
+ * block ("KV-outer": each K/V block gathers its queries), plus a work list for the attention.
+ *
+ * The result lives in ONE caller-allocated device buffer `kv2q` of layout.total_bytes bytes,
+ * described by a host-side msa_kv2q_layout filled by msa_kv2q_layout_get(). Arrays in it:
+ *   offsets      int32 [H_kv][nb + 1]  CSR row pointers per group; offsets[r][0] = 0
+ *   entries      int32 [H_kv][N * k]   list of block b of group r = entries[r][offsets[r][b] ..
+ *                                      offsets[r][b+1]), rows ascending, each entry i*k + slot
+ *                                      (slot = rank of b in row i's ascending set)
+ *   items        msa_work_item [max_items]  ordered window-major: all items whose rows lie in
+ *                                      query window w (rows [w*window, (w+1)*window)) precede
+ *                                      those of window w+1; inside a window, by (r, b). An item
+ *                                      covers at most `chunk` consecutive entries of one list.
+ *   window_items int32 [n_windows + 1] first item of each window; the last value is the count
+ *   (plus internal per-(r, b, window) counts used while building)
+ * window = 0 / chunk = 0 select the defaults (2048 rows per window, chunk = window).
+ * ------------------------------------------------------------------------------------------ */
+typedef struct {
+    int32_t r;     /* GQA group */
+    int32_t b;     /* KV block */
+    int32_t start; /* first entry, index into entries[r] */
+    int32_t len;   /* number of entries */
+} msa_work_item;
+
+typedef struct {
+    int64_t N;
+    int32_t H_kv, B_k, k, nb;
+    int32_t window, chunk, n_windows;
+    int64_t max_items;
+    size_t offsets, entries, items, window_items, counts, bases; /* byte offsets into the buffer */
+    size_t total_bytes;
+} msa_kv2q_layout;
+
+MSA_API msa_status msa_kv2q_layout_get(int64_t N, int H_kv, int B_k, int k, int window, int chunk, msa_kv2q_layout* layout);
+
+MSA_API size_t msa_build_kv2q_workspace_size(const msa_kv2q_layout* layout);
+
+/*   block_idx : [H_kv, N, k] int32 as written by msa_index_topk (ascending, -1 padded)
+ *   layout    : host struct from msa_kv2q_layout_get with the same N, H_kv, B_k, k
+ *   kv2q      : device buffer of layout->total_bytes bytes, filled by this call */
+MSA_API msa_status msa_build_kv2q(const int32_t* block_idx, const msa_kv2q_layout* layout, void* kv2q, void* workspace,
+                          size_t workspace_bytes, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Main Branch: exact block-sparse causal attention, KV-outer, two-stage      [EXPL 05-2, ABS]
+ *
+ * For row i, head h (group r = floor(h / G)) and T = {j <= i : block(j) in set(i, r)}:
+ *   out[i, h] = sum_{j in T} softmax_T(q[i,h] . k[j,r] / sqrt(d_h)) v[j, r]
+ *   lse[i, h] = log sum_{j in T} exp(q[i,h] . k[j,r] / sqrt(d_h))   (natural log, scaled logits)
+ * Stage 1 walks the work list: each item stages its K/V block once and gathers 128/G query
+ * rows x G heads per 128-row tensor-core tile, writing a partial (normalised output, lse) per
+ * (row, head, slot). Stage 2 merges the <= k partials of each (row, head) through their lse.
+ *
+ *   q        : [N, H_q, d_h] bf16;   k, v : [N, H_kv, d_h] bf16  (16-byte aligned)
+ *   block_idx: [H_kv, N, k] int32 (msa_index_topk output)
+ *   layout, kv2q : a built inversion, or both NULL to build it inside the workspace
+ *   out      : [N, H_q, d_h] bf16 out;  lse : [N, H_q] fp32 out, or NULL
+ *   workspace: >= msa_sparse_prefill_workspace_size(..., max_rows_per_pass, internal_kv2q).
+ *              Partials need about H_q * k * (2*d_h + 4) bytes per query row; when the workspace
+ *              holds fewer rows than N the call processes the query windows in passes.
+ * ------------------------------------------------------------------------------------------ */
+MSA_API size_t msa_sparse_prefill_workspace_size(int64_t N, int H_q, int H_kv, int d_h, int B_k, int k,
+                                         int64_t max_rows_per_pass, int internal_kv2q);
+
+MSA_API msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* k, const msa_bf16* v, int64_t N, int H_q, int H_kv,
+                              int d_h, int B_k, int kk, const int32_t* block_idx, const msa_kv2q_layout* layout,
+                              const void* kv2q, msa_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
+                              msa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Decode: one query token per sequence against a KV cache                  [ABS, EXPL Fig. 4]
+ *
+ * Sequence beta holds lens[beta] cached tokens (the current token included) and its query sits
+ * at position i = lens[beta] - 1; selection and attention are those of prefill row i of that
+ * sequence. The index scores stream over the k_idx cache split across CTAs, per-lane register
+ * Top-k lists are merged with warp shuffles, then split attention over the k selected blocks is
+ * merged through the lse like prefill.
+ *
+ *   q       : [B, H_q, d_h] bf16;  q_idx : [B, H_kv, d_idx] bf16
+ *   k_cache, v_cache : [B, L_max, H_kv, d_h] bf16;  k_idx_cache : [B, L_max, H_kv, d_idx] bf16
+ *   lens    : [B] int32 device array, 1 <= lens[beta] <= L_max (checked on the device; a bad
+ *             length sets MSA_ERR_DEVICE_CHECK and that sequence's output is left unwritten)
+ *   out     : [B, H_q, d_h] bf16 out;  lse : [B, H_q] fp32 out or NULL
+ *   block_idx_out : [B, H_kv, k] int32 out or NULL (the selections)
+ * ------------------------------------------------------------------------------------------ */
+MSA_API size_t msa_sparse_decode_workspace_size(int B, int64_t L_max, int H_q, int H_kv, int d_h, int d_idx, int B_k, int k);
+
+MSA_API msa_status msa_sparse_decode(const msa_bf16* q, const msa_bf16* q_idx, const msa_bf16* k_cache,
+                             const msa_bf16* v_cache, const msa_bf16* k_idx_cache, const int32_t* lens, int B,
+                             int64_t L_max, int H_q, int H_kv, int d_h, int d_idx, int B_k, int k, msa_bf16* out,
+                             float* lse, int32_t* block_idx_out, void* workspace, size_t workspace_bytes,
+                             msa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Tracing (measurement support; no counterpart on the pages)
+ *
+ * msa_trace_set() installs a caller-owned record: while installed, every entry point records
+ * events[2j] / events[2j+1] (caller-created cudaEvent_t handles) on its stream immediately
+ * before / after its j-th traced kernel and stores that kernel's id in kernel_ids[j]; `count`
+ * advances by 2 per traced kernel and recording stops silently at `capacity`. NULL uninstalls.
+ * Process-wide and not thread-safe: one tracing caller at a time. msa_launch_count() returns the
+ * number of kernels this library has launched in the process (for launch accounting).
+ * ------------------------------------------------------------------------------------------ */
+typedef enum {
+    MSA_KERNEL_INDEX_TOPK = 1, /* fused index score + max-pool + Top-k                         */
+    MSA_KERNEL_KV2Q = 2,       /* whole KV->Q inversion (count, scans, scatter, work list)      */
+    MSA_KERNEL_ATTN = 3,       /* KV-outer attention, stage 1 (one per pass)                    */
+    MSA_KERNEL_COMBINE = 4,    /* LSE combine, stage 2 (one per pass)                           */
+    MSA_KERNEL_DEC_POOL = 5,   /* decode index scores + max-pool                                */
+    MSA_KERNEL_DEC_TOPK = 6,   /* decode Top-k warp merge                                       */
+    MSA_KERNEL_DEC_ATTN = 7,   /* decode split attention                                        */
+    MSA_KERNEL_DEC_COMBINE = 8 /* decode LSE combine                                            */
+} msa_kernel_id;
+
+typedef struct {
+    void** events;   /* cudaEvent_t handles, two per traced kernel */
+    int capacity;    /* number of handles in events */
+    int count;       /* handles used so far (written by the library) */
+    int* kernel_ids; /* [capacity / 2] msa_kernel_id of each traced kernel (written) */
+} msa_trace;
+
+MSA_API void msa_trace_set(msa_trace* trace);
+
+MSA_API uint64_t msa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */
