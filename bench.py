@@ -46,6 +46,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-oracle sample time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows-per-pass", type=int, default=0, help="cap the prefill partial buffer (0 = whole N)")
     return ap.parse_args()
 
 
@@ -132,7 +133,7 @@ class ClockSampler:
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -201,8 +202,8 @@ def gpu_arm(args, rank, world):
     kv = msa.KV2Q(L, torch.empty(L.total_bytes, dtype=torch.uint8, device=dev))
     ws_kv = torch.empty(msa.api.lib.msa_build_kv2q_workspace_size(msa.api.ctypes.byref(L)), dtype=torch.uint8,
                         device=dev)
-    ws_pf = torch.empty(msa.msa_sparse_prefill_workspace_size(N, H_q, H_kv, d_h, cfg.B_k, k), dtype=torch.uint8,
-                        device=dev)
+    ws_pf = torch.empty(msa.msa_sparse_prefill_workspace_size(N, H_q, H_kv, d_h, cfg.B_k, k, args.rows_per_pass),
+                        dtype=torch.uint8, device=dev)
     out = torch.empty_like(t["q"])
     lse = torch.empty((N, H_q), dtype=torch.float32, device=dev)
     ws_idx = torch.empty(256, dtype=torch.uint8, device=dev)
