@@ -7,7 +7,10 @@
 //   M = max_s lse_s,  w_s = exp(lse_s - M),  L = sum_s w_s
 //   out[i, h] = sum_s (w_s / L) * o_s,        lse[i, h] = M + log(L)
 // Slots are merged in the fixed order 0..n_sel-1, so the result is deterministic.
-// One CTA per row: the row's partials are a contiguous [k][H_q][d_h] slab read with 16-byte loads.
+//
+// Partials are laid out [row][slot][d_h/8][H_q][8] (bf16) and [row][slot][H_q] (fp32 lse). One CTA
+// per row reads the row's contiguous slabs with 16-byte loads (all slots of a unit in flight at
+// once), and stages the merged row in shared memory so the output row is written contiguously.
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -20,7 +23,9 @@ constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 {
-    extern __shared__ float wsm[]; // [k][H_q] normalised weights
+    extern __shared__ __align__(16) uint8_t csm[];
+    float* wsm = reinterpret_cast<float*>(csm);                                 // [k][H_q] weights
+    uint4* obuf = reinterpret_cast<uint4*>(csm + align_up_dev(a.k * a.H_q * 4)); // [H_q][d_h/8] swizzled
     const int64_t i = a.row0 + blockIdx.x;
     const int64_t prow = blockIdx.x;
     const int n_sel = a.nsel ? a.nsel[prow] : (int)min((int64_t)a.k, i / a.local_of_row_div + 1);
@@ -40,22 +45,28 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
         if (a.lse) a.lse[i * a.H_q + h] = M + logf(L);
     }
     __syncthreads();
-    const int units = a.H_q * a.d_h / 8; // 8 bf16 per 16-byte unit
+    const int NC = a.d_h / 8;     // 16-byte units per head
+    const int units = a.H_q * NC; // per slot
     const uint4* op = reinterpret_cast<const uint4*>(a.o_part + prow * a.k * a.H_q * (int64_t)a.d_h);
-    uint4* dst = reinterpret_cast<uint4*>(a.out + i * a.H_q * (int64_t)a.d_h);
     for (int u = threadIdx.x; u < units; u += blockDim.x) {
-        const int h = (u * 8) / a.d_h;
+        const int c = u / a.H_q, h = u - c * a.H_q;
+        uint4 v[kMaxK];
+#pragma unroll
+        for (int s = 0; s < kMaxK; ++s)
+            if (s < n_sel) v[s] = op[(int64_t)s * units + u];
         float acc[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-        for (int s = 0; s < n_sel; ++s) {
-            const float w = wsm[s * a.H_q + h];
-            const uint4 v = op[(int64_t)s * units + u];
-            const uint32_t x[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                acc[2 * q] = fmaf(w, __uint_as_float(x[q] << 16), acc[2 * q]);
-                acc[2 * q + 1] = fmaf(w, __uint_as_float(x[q] & 0xFFFF0000u), acc[2 * q + 1]);
+        for (int s = 0; s < kMaxK; ++s) {
+            if (s < n_sel) {
+                const float w = wsm[s * a.H_q + h];
+                const uint32_t x[4] = {v[s].x, v[s].y, v[s].z, v[s].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[2 * q] = fmaf(w, __uint_as_float(x[q] << 16), acc[2 * q]);
+                    acc[2 * q + 1] = fmaf(w, __uint_as_float(x[q] & 0xFFFF0000u), acc[2 * q + 1]);
+                }
             }
         }
         uint32_t o[4];
@@ -65,7 +76,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
             asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(acc[2 * q]), "f"(acc[2 * q + 1]));
             o[q] = r;
         }
-        dst[u] = make_uint4(o[0], o[1], o[2], o[3]);
+        obuf[h * NC + (c ^ (h & (NC - 1)))] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    __syncthreads();
+    uint4* dst = reinterpret_cast<uint4*>(a.out + i * a.H_q * (int64_t)a.d_h);
+    for (int u = threadIdx.x; u < units; u += blockDim.x) {
+        const int h = u / NC, c = u - h * NC;
+        dst[u] = obuf[h * NC + (c ^ (h & (NC - 1)))];
     }
 }
 
@@ -74,7 +91,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s)
 {
     if (a.n_rows <= 0) return cudaSuccess;
-    const size_t smem = (size_t)a.k * a.H_q * sizeof(float);
+    const size_t smem = align_up((size_t)a.k * a.H_q * sizeof(float), 16) + (size_t)a.H_q * a.d_h * 2;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
     combine_kernel<<<(unsigned)a.n_rows, kCombineThreads, smem, s>>>(a);
     note_launch(1);
     return cudaGetLastError();

@@ -30,6 +30,7 @@ __device__ __forceinline__ void report_error(int* word, int code, int detail)
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ inline int align_up_dev(int x) { return (x + 15) & ~15; }
 
 // Opt-in per-kernel event tracing and the launch counter (msa_trace_set / msa_launch_count).
 void trace_begin(cudaStream_t s);
@@ -76,6 +77,8 @@ struct AttnArgs {
     int w0, w1;                 // windows of this pass
     int64_t row0;               // first row of the pass (= w0 * window)
     int64_t rows_pass;          // rows the partial buffers hold
+    long long* timeline;        // optional: CTA 0 records clock64 per tile event (nullptr = off)
+    int timeline_tiles;         // capacity in tiles (8 events per tile)
     uint16_t* o_part;           // [rows][k][H_q][d_h]
     float* lse_part;            // [rows][k][H_q]
     int* err;

@@ -356,6 +356,8 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
         a.w1 = (int)w1;
         a.row0 = w0 * L->window;
         a.rows_pass = rows_pass;
+        a.timeline = nullptr;
+        a.timeline_tiles = 0;
         a.o_part = o_part;
         a.lse_part = lse_part;
         a.err = (int*)workspace;
