@@ -47,6 +47,7 @@ SIGNATURES = [
     ("msa_kv2q_layout_get", _int, [_i64, _int, _int, _int, _int, _int, _LP]),
     ("msa_build_kv2q_workspace_size", _sz, [_LP]),
     ("msa_build_kv2q", _int, [_vp, _LP, _vp, _vp, _sz, _vp]),
+    ("msa_build_kv2q_static", _int, [_vp, _LP, _vp, _vp]),
     ("msa_sparse_prefill_workspace_size", _sz, [_i64, _int, _int, _int, _int, _int, _i64, _int]),
     ("msa_sparse_prefill", _int, [_vp, _vp, _vp, _i64, _int, _int, _int, _int, _int, _vp, _LP, _vp, _vp, _vp, _vp,
                                   _sz, _vp]),

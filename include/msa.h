@@ -142,6 +142,27 @@ MSA_API size_t msa_build_kv2q_workspace_size(const msa_kv2q_layout* layout);
 MSA_API msa_status msa_build_kv2q(const int32_t* block_idx, const msa_kv2q_layout* layout, void* kv2q, void* workspace,
                           size_t workspace_bytes, msa_stream_t stream);
 
+/*
+ * msa_build_kv2q_static: the same inversion as msa_build_kv2q, for callers that cannot allocate
+ * device memory. The pages have no counterpart; this is an interface variant, not a step of the
+ * method. Typical such callers are plug-ins handed only their input and output buffers by a host
+ * framework that owns every device allocation, and latency-critical loops where a cudaMalloc or
+ * cudaFree would synchronise the device.
+ *   - No workspace argument and no allocation: the scratch (device error word + scan partials)
+ *     is a fixed 1 MiB array of this library (a file-scope __device__ array), held by every GPU
+ *     that loads the library until the process exits. The caller still passes block_idx, the
+ *     layout and the kv2q output buffer, exactly as for msa_build_kv2q.
+ *   - The first call on a device looks up the array's device address on that device (it must be
+ *     the current device); make that first call before any stream capture.
+ *   - Layouts whose scratch would exceed 1 MiB are rejected with MSA_ERR_WORKSPACE (every shape
+ *     this build supports fits: the scan needs one int32 per 1024 (group, block, window) counters).
+ *   - All calls share the one array: calls whose work overlaps on the GPU (other streams, other
+ *     threads) race on it. The error word is cleared at the start of every call; the variant
+ *     does not expose it, so out-of-range block ids are skipped without a report.
+ */
+MSA_API msa_status msa_build_kv2q_static(const int32_t* block_idx, const msa_kv2q_layout* layout, void* kv2q,
+                                         msa_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Main Branch: exact block-sparse causal attention, KV-outer, two-stage      [EXPL 05-2, ABS]
  *
