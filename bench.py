@@ -15,7 +15,6 @@ on a bounded sample of the same workload, and prints the same metric.
 from __future__ import annotations
 
 import argparse
-import datetime
 import json
 import os
 import statistics
@@ -29,7 +28,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from block_sparse_long_idx_b200 import roofline, synth  # noqa: E402
+from block_sparse_long_idx_b200 import replicas, roofline, synth  # noqa: E402
 
 METRIC = "MSA prefill tokens/s @N=128K (64q/4kv heads), decode tok/s; % of roofline"
 UNIT = "tokens/s"
@@ -184,8 +183,8 @@ def gpu_arm(args, rank, world):
     dev = torch.device("cuda", local)
     peaks = load_peaks()
     cfg = synth.PREFILL_CONFIGS[args.workload]
-    cfg = cfg.with_(seed=cfg.seed + 1000 * rank)  # independent sequence per rank
-    dcfg = None if args.no_decode else synth.DECODE64.with_(seed=synth.DECODE64.seed + 1000 * rank)
+    cfg = cfg.with_(seed=replicas.replica_seed(cfg.seed, rank))  # independent sequence per rank
+    dcfg = None if args.no_decode else synth.DECODE64.with_(seed=replicas.replica_seed(synth.DECODE64.seed, rank))
 
     host = synth.prefill_inputs(cfg)
     cpu_base = None
@@ -268,11 +267,7 @@ def gpu_arm(args, rank, world):
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
     kern = trace.durations()
 
-    # max over ranks
-    tt = torch.tensor([sum(pf_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    pf_total, dec_total = tt.tolist()
+    pf_total, dec_total = replicas.max_over_ranks([sum(pf_ms), sum(dec_ms)], device=dev)
 
     # end-to-end through the public API with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -294,16 +289,15 @@ def gpu_arm(args, rank, world):
             e1.record()
             torch.cuda.synchronize()
             tot += e0.elapsed_time(e1)
-        te = torch.tensor([tot], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * N * args.e2e_steps / (te.item() / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        (te,) = replicas.max_over_ranks([tot], device=dev)
+        e2e = {"value": replicas.aggregate_rate(N * args.e2e_steps, world, te / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
                "note": "prefill through the public API: pinned host inputs copied in, out copied back"}
 
     if rank != 0:
         return
-    value = world * N * args.steps / (pf_total / 1000.0)
+    value = replicas.aggregate_rate(N * args.steps, world, pf_total / 1000.0)
     kstats = {}
     fl_main = roofline.main_branch_flops(N, H_q, d_h, k, cfg.B_k)
     fl_idx = roofline.index_branch_flops(N, H_kv, d_idx)
@@ -346,15 +340,12 @@ def gpu_arm(args, rank, world):
 
 def main():
     args = parse_args()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    rank, world, _ = replicas.rank_info()
     if args.impl == "reference":
         reference_arm(args, rank)
         return
     if world > 1:
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        replicas.init("nccl", timeout_s=300)
     try:
         gpu_arm(args, rank, world)
     finally:

@@ -310,17 +310,17 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
     size_t used = kErrBytes;
     const void* kv = kv2q;
     cudaStream_t s = (cudaStream_t)stream;
-    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    // every size check happens before anything is enqueued
+    void* kvbuf = nullptr;
+    void* kvtmp = nullptr;
     if (!L) {
         msa_kv2q_layout_get(N, H_kv, B_k, k, 0, 0, &Lint);
         L = &Lint;
         const size_t need = align_up(L->total_bytes, 256) + align_up(kv2q_internal_tmp(*L), 256);
         if (workspace_bytes < used + need) return MSA_ERR_WORKSPACE;
-        void* kvbuf = ws + used;
-        void* tmp = ws + used + align_up(L->total_bytes, 256);
+        kvbuf = ws + used;
+        kvtmp = ws + used + align_up(L->total_bytes, 256);
         used += need;
-        msa_status st = build_kv2q_impl(block_idx, L, kvbuf, (int*)workspace, tmp, s);
-        if (st != MSA_OK) return st;
         kv = kvbuf;
     }
     // rows of partials the remaining workspace holds, in whole windows
@@ -340,6 +340,11 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
         !make_map_3d(&vmap, v, d_h, H_kv, N, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B))
         return MSA_ERR_INVALID_ARG;
 
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    if (kvbuf) {
+        msa_status st = build_kv2q_impl(block_idx, L, kvbuf, (int*)workspace, kvtmp, s);
+        if (st != MSA_OK) return st;
+    }
     const uint8_t* kvb = (const uint8_t*)kv;
     for (int64_t w0 = 0; w0 < L->n_windows; w0 += wins_per_pass) {
         const int64_t w1 = w0 + wins_per_pass < L->n_windows ? w0 + wins_per_pass : L->n_windows;

@@ -1,0 +1,108 @@
+"""The C ABI on the host, no GPU needed: the library loads, exports every symbol include/msa.h declares,
+rejects bad arguments with the documented status before touching the device, sizes its workspaces,
+and honours host-side fault injection."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA = 0, 1, 2, 3, 4
+P, P2, WS = 0x100000, 0x200000, 0x300000  # fake, suitably aligned device addresses (never dereferenced)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MSA_API\s+[\w\s\*]*?\b(msa_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def msa():
+    from block_sparse_long_idx_b200 import build
+
+    if not os.path.exists(build.LIB):
+        build.build()
+    import block_sparse_long_idx_b200 as m
+
+    return m
+
+
+def test_every_declared_symbol_is_exported(msa):
+    names = declared_symbols()
+    assert len(names) >= 15
+    raw = ctypes.CDLL(msa.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    bound = {s[0] for s in msa.SIGNATURES}
+    assert set(names) <= bound, set(names) - bound
+
+
+def test_status_strings(msa):
+    assert msa.status_string(0) == "MSA_OK"
+    assert msa.status_string(3) == "MSA_ERR_WORKSPACE"
+    assert msa.status_string(6) == "MSA_ERR_DEVICE_CHECK"
+
+
+def test_index_topk_validation(msa):
+    f = msa.lib.msa_index_topk
+    assert f(None, P2, 1024, 2, 64, 128, 4, P, WS, 256, None) == INVALID        # null input
+    assert f(P + 2, P2, 1024, 2, 64, 128, 4, P, WS, 256, None) == INVALID       # misaligned
+    assert f(P, P2, 0, 2, 64, 128, 4, P, WS, 256, None) == INVALID              # N < 1
+    assert f(P, P2, 1024, 2, 48, 128, 4, P, WS, 256, None) == UNSUPPORTED       # d_idx
+    assert f(P, P2, 1024, 2, 64, 64, 4, P, WS, 256, None) == UNSUPPORTED        # B_k != 128
+    assert f(P, P2, 1024, 2, 64, 128, 17, P, WS, 256, None) == UNSUPPORTED      # k > 16
+    assert f(P, P2, 1024, 2, 64, 128, 4, P, WS, 16, None) == WORKSPACE          # workspace too small
+
+
+def test_layout_and_workspace_sizes(msa):
+    L = msa.msa_kv2q_layout_get(131072, 4, 128, 16)
+    assert L.nb == 1024 and L.n_windows == 64 and L.window == 2048 and L.chunk == 512
+    assert L.entries > L.offsets and L.total_bytes > L.bases
+    with pytest.raises(msa.MsaError):
+        msa.msa_kv2q_layout_get(1000, 2, 128, 4, window=100)    # window not a multiple of B_k
+    ws = msa.api.lib.msa_sparse_prefill_workspace_size(131072, 64, 4, 128, 128, 16, 0, 0)
+    assert ws > 131072 * 16 * 64 * 260                           # holds every partial of one pass
+    ws8 = msa.api.lib.msa_sparse_prefill_workspace_size(131072, 64, 4, 128, 128, 16, 8192, 0)
+    assert ws8 < ws / 10                                         # a pass cap shrinks it
+    assert msa.api.lib.msa_sparse_decode_workspace_size(64, 131072, 64, 4, 128, 64, 128, 16) > 0
+
+
+def test_prefill_and_decode_validation(msa):
+    L = msa.msa_kv2q_layout_get(1024, 2, 128, 4)
+    pf = msa.lib.msa_sparse_prefill
+    # H_q % H_kv != 0
+    assert pf(P, P, P, 1024, 6, 4, 128, 128, 4, P, None, None, P, None, WS, 1 << 30, None) == INVALID
+    # d_h unsupported
+    assert pf(P, P, P, 1024, 8, 2, 96, 128, 4, P, None, None, P, None, WS, 1 << 30, None) == UNSUPPORTED
+    # layout given without buffer
+    assert pf(P, P, P, 1024, 8, 2, 128, 128, 4, P, ctypes.byref(L), None, P, None, WS, 1 << 30, None) == INVALID
+    # workspace too small for one window of partials
+    assert pf(P, P, P, 1024, 8, 2, 128, 128, 4, P, ctypes.byref(L), P2, P, None, WS, 1024, None) == WORKSPACE
+    dec = msa.lib.msa_sparse_decode
+    args = [P, P, P, P, P, P, 4, 4096, 64, 4, 128, 64, 128, 16, P, None, None, WS, 1 << 30, None]
+    bad = list(args)
+    bad[5] = None                                                # lens missing
+    assert dec(*bad) == INVALID
+    g32 = list(args)
+    g32[8] = 128                                                 # G = 32 > 16 for decode
+    assert dec(*g32) == UNSUPPORTED
+    small = list(args)
+    small[18] = 256
+    assert dec(*small) == WORKSPACE
+
+
+def test_host_fault_injection():
+    """MSA_FAULT_INJECT=<entry point> makes that call fail as a launch failure would, before enqueueing."""
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "import block_sparse_long_idx_b200 as m\n"
+        "r = m.lib.msa_index_topk(%d, %d, 1024, 2, 64, 128, 4, %d, %d, 256, None)\n"
+        "print('STATUS', r)\n" % (ROOT, P, P2, P, WS))
+    env = dict(os.environ, MSA_FAULT_INJECT="msa_index_topk")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert "STATUS 4" in out.stdout, out.stdout + out.stderr

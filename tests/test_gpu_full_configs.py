@@ -1,0 +1,100 @@
+"""GPU parity at the full workload sizes, in the launch configuration bench.py times (default query
+windows and chunks): 32K, the 128K planted sequence, 1M (4096 sampled rows, as stated for 1M-token
+configs) and the 64-sequence decode batch.
+
+Sampled rows are checked against the oracle (selections bit-exact, outputs within tolerance);
+properties that hold at any size are checked on every row: each selected set contains its local
+block, has min(k, local+1) ascending visible blocks, and the KV->Q lists are exactly the inversion
+of the selections."""
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import block_sparse_long_idx_b200 as msa  # noqa: E402
+import oracle  # noqa: E402
+from block_sparse_long_idx_b200 import synth  # noqa: E402
+from tests.gpu_util import (assert_lse_close, assert_out_close, assert_selection_equal, bf16_to_f64,  # noqa: E402
+                            dev)
+
+
+def check_selection_properties(bi: np.ndarray, B_k: int):
+    H_kv, N, k = bi.shape
+    local = (np.arange(N) // B_k)[None, :, None]
+    valid = bi >= 0
+    n = valid.sum(-1)
+    want_n = np.minimum(k, np.arange(N) // B_k + 1)[None, :]
+    assert (n == want_n).all(), "set sizes"
+    assert (valid[..., :-1] >= valid[..., 1:]).all(), "-1 padding must trail"
+    assert ((bi == local).any(-1)).all(), "local block missing"
+    assert ((bi <= local) | ~valid).all(), "invisible block selected"
+    d = np.diff(np.where(valid, bi, np.iinfo(np.int32).max), axis=-1)
+    assert (d[valid[..., 1:]] > 0).all(), "not strictly ascending"
+
+
+def check_inversion(kv, bi: np.ndarray):
+    H_kv, N, k = bi.shape
+    off = kv.offsets().cpu().numpy().astype(np.int64)
+    ent = kv.entries().cpu().numpy()
+    nb = off.shape[1] - 1
+    for r in range(H_kv):
+        flat = bi[r].reshape(-1)
+        idx = np.nonzero(flat >= 0)[0]
+        order = np.argsort(flat[idx], kind="stable")  # by block, rows ascending within a block
+        want_ent = idx[order].astype(np.int32)          # flat index i*k + slot
+        want_off = np.concatenate([[0], np.cumsum(np.bincount(flat[idx], minlength=nb))])
+        assert np.array_equal(off[r], want_off), f"offsets of group {r}"
+        assert np.array_equal(ent[r, :len(want_ent)], want_ent), f"entries of group {r}"
+
+
+def run_prefill(cfg, n_rows, rows_per_pass=0):
+    inp = synth.prefill_inputs(cfg)
+    t = {n: dev(a) for n, a in inp.items()}
+    bi = msa.msa_index_topk(t["q_idx"], t["k_idx"], cfg.B_k, cfg.k)
+    kv = msa.msa_build_kv2q(bi, cfg.B_k)
+    ws = torch.empty(msa.msa_sparse_prefill_workspace_size(cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.B_k, cfg.k,
+                                                           rows_per_pass), dtype=torch.uint8, device="cuda")
+    out, lse = msa.msa_sparse_prefill(t["q"], t["k"], t["v"], bi, kv, workspace=ws)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(ws) == 0
+    del t
+    bih = bi.cpu().numpy()
+    check_selection_properties(bih, cfg.B_k)
+    check_inversion(kv, bih)
+    rows = synth.sample_rows(cfg.N, cfg.B_k, n_rows, cfg.seed)
+    sel, want, want_lse = oracle.prefill_rows(inp, rows, cfg.B_k, cfg.k)
+    assert_selection_equal(np.ascontiguousarray(bih[:, rows, :]), np.ascontiguousarray(sel.transpose(1, 0, 2)),
+                           rows)
+    got = bf16_to_f64(out[torch.from_numpy(rows).cuda()])
+    assert_out_close(got, want)
+    assert_lse_close(lse[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64), want_lse)
+
+
+def test_prefill_32k():
+    run_prefill(synth.P32K, 512)
+
+
+def test_prefill_128k_planted():
+    run_prefill(synth.P128K, 512)
+
+
+def test_prefill_1m_sampled():
+    """1M tokens, processed in passes of 131072 query rows (the partial buffer of one pass is ~35 GB)."""
+    run_prefill(synth.P1M, 4096, rows_per_pass=131072)
+
+
+def test_decode_64_sequences():
+    cfg = synth.DECODE64
+    inp = synth.decode_inputs(cfg)
+    t = {n: dev(a) for n, a in inp.items()}
+    out, lse, bi = msa.msa_sparse_decode(t["q"], t["q_idx"], t["k_cache"], t["v_cache"], t["k_idx_cache"], t["lens"],
+                                         cfg.B_k, cfg.k)
+    torch.cuda.synchronize()
+    sel, want, want_lse = oracle.decode(inp, cfg.B_k, cfg.k)
+    assert np.array_equal(bi.cpu().numpy(), sel), "decode selection differs"
+    assert_out_close(bf16_to_f64(out), want)
+    assert_lse_close(lse.cpu().numpy().astype(np.float64), want_lse)
