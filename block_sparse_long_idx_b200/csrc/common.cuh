@@ -78,7 +78,7 @@ struct AttnArgs {
     int64_t row0;               // first row of the pass (= w0 * window)
     int64_t rows_pass;          // rows the partial buffers hold
     long long* timeline;        // optional: CTA 0 records clock64 per tile event (nullptr = off)
-    int timeline_tiles;         // capacity in tiles (8 events per tile)
+    int timeline_tiles;         // capacity in tiles (16 event slots per tile)
     uint16_t* o_part;           // [rows][k][H_q][d_h]
     float* lse_part;            // [rows][k][H_q]
     int* err;

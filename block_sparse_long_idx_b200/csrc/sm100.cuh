@@ -63,6 +63,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait without a suspend hint: for the thread on the critical path (the MMA issuer), which
+// must notice a completed phase as soon as possible.
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete. Gives up after `limit` clock cycles and
 // returns false; every caller turns that into an error status instead of spinning forever.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit)
@@ -255,6 +268,23 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+// 32 columns from r[OFF .. OFF+31] of a larger register array.
+template <int OFF, int N>
+__device__ __forceinline__ void tmem_st32_at(uint32_t taddr, const uint32_t (&r)[N])
+{
+    static_assert(OFF + 32 <= N, "range");
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[OFF + 0]), "r"(r[OFF + 1]), "r"(r[OFF + 2]), "r"(r[OFF + 3]), "r"(r[OFF + 4]), "r"(r[OFF + 5]),
+        "r"(r[OFF + 6]), "r"(r[OFF + 7]), "r"(r[OFF + 8]), "r"(r[OFF + 9]), "r"(r[OFF + 10]), "r"(r[OFF + 11]),
+        "r"(r[OFF + 12]), "r"(r[OFF + 13]), "r"(r[OFF + 14]), "r"(r[OFF + 15]), "r"(r[OFF + 16]), "r"(r[OFF + 17]),
+        "r"(r[OFF + 18]), "r"(r[OFF + 19]), "r"(r[OFF + 20]), "r"(r[OFF + 21]), "r"(r[OFF + 22]), "r"(r[OFF + 23]),
+        "r"(r[OFF + 24]), "r"(r[OFF + 25]), "r"(r[OFF + 26]), "r"(r[OFF + 27]), "r"(r[OFF + 28]), "r"(r[OFF + 29]),
+        "r"(r[OFF + 30]), "r"(r[OFF + 31])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait()
 {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -297,6 +327,23 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     return true;
 }
 
+// wait_or_abort for the MMA issuer: busy-polls (test_wait) instead of sleeping.
+__device__ __forceinline__ bool poll_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                              int site, long long limit)
+{
+    if (mbar_poll(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_poll(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > limit) {
+            if (atomicCAS(err, 0, 5 /* MSA_ERR_TIMEOUT */) == 0) err[1] = site;
+            *abort_flag = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
 __device__ __forceinline__ float ex2_approx(float x)
 {
     float y;
@@ -315,6 +362,18 @@ template <int N>
 __device__ __forceinline__ void reg_alloc()
 {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Set a warpgroup's register count to N from the LAUNCH count the kernel was compiled for:
+// setmaxnreg.inc may only raise and setmaxnreg.dec may only lower the current count.
+template <int N, int LAUNCH>
+__device__ __forceinline__ void reg_set()
+{
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+    if constexpr (N > LAUNCH)
+        reg_alloc<N>();
+    else if constexpr (N < LAUNCH)
+        reg_dealloc<N>();
 }
 
 __device__ __forceinline__ float max3f(float a, float b, float c)

@@ -8,17 +8,26 @@
 //   S = Q K^T                         tcgen05.mma, A = Q (smem), B = K (smem), D in TMEM
 //   P = exp(S*scale - rowmax)         softmax warps, thread = TMEM lane = tile row; the causal mask
 //                                     only applies to rows whose own block is b; P goes back to
-//                                     TMEM as bf16 over the S columns
+//                                     TMEM as bf16 over the first 64 S columns
 //   O = P V                           tcgen05.mma, A = P (TMEM), B = V (smem, MN-major)
 //   partial[p, slot, h] = O / rowsum, lse = rowmax*scale + log(rowsum)
 // A work item covers one KV block only, so no running-max rescaling is needed. Stage 2
 // (combine.cu) merges the <= k partials of every (row, head) through their lse.
 //
-// Roles (384 threads): warp 0 = K/V TMA producer, warp 1 = MMA issuer + TMEM owner, warp 2 = Q
-// gather (one TMA box per position, issued by the 32 lanes in parallel), warps 4-7 and 8-11 =
-// softmax + epilogue for even and odd tiles. TMEM: S/P of tile buffer i at columns [128 i, +128),
-// O of buffer i at [256 + 128 i, +d_h). Barriers per buffer: s_full (S written), p_full (P
-// written), o_full (O written, which also frees S/P), o_free (epilogue has read O).
+// Roles (512 threads, four warpgroups):
+//   WG0: warp 0 = K/V TMA producer, warp 1 = S issuer + TMEM owner, warp 2 = Q gather (one TMA
+//        box per position, issued by the 32 lanes in parallel), warp 3 = PV issuer
+//   WG1, WG2: softmax of even / odd tiles
+//   WG3: epilogue of every tile (O / rowsum -> partial slot)
+// TMEM (512 columns): two 128-column S/P regions A[t % 2] at columns 0 and 128 (S, then P in
+// columns 0-63) and two output regions O[t % 2] at columns 256 and 384. Two threads issue the
+// MMAs, so neither's polling leaves the tensor pipe idle: the S issuer issues S(t) once PV(t-2)
+// has consumed P(t-2) (region A[t % 2] free); the PV issuer issues PV(t) once P(t) is written and
+// the epilogue of t-2 has read O[t % 2], which leaves the epilogue a full tile of slack.
+// Barriers: s_full[2], p_full[2], pv_done[2] per S/P region; o_full[2], o_free[2] per O region;
+// ml_full[4] hands each tile's row max and row sum from the softmax to the epilogue through shared
+// memory (slot t % 4, rewritten by the softmax of t+4, which needs S(t+4), which needs PV(t+2),
+// which needs the epilogue of t to have read O).
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -33,24 +42,32 @@ struct AttnCfg {
     static constexpr int NKC = DH / 64;          // 64-column (128-byte) chunks
     static constexpr int CHUNK = 128 * 128;      // bytes per chunk of a 128-row tile
     static constexpr int TILE = NKC * CHUNK;     // Q, K or V tile bytes
-    static constexpr int NQ = 3;                 // Q stages
+    static constexpr int NQ = 2;                 // Q stages
     static constexpr int SMEM = 1024 + NQ * TILE + 4 * TILE;
 };
 
 struct AttnShared {
     uint64_t kv_full[2], kv_empty[2];
-    uint64_t q_full[3], q_empty[3];
-    uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
-    uint64_t done;
+    uint64_t q_full[2], q_empty[2];
+    uint64_t s_full[2], p_full[2], pv_done[2];
+    uint64_t o_full[2], o_free[2];
+    uint64_t ml_full[4];
+    uint64_t done, done2;
+    float2 ml[4][128]; // (row max of the raw scores, row sum of exp) per tile slot and row
     uint32_t tmem_base;
     int abort_flag;
 };
 
 constexpr uint32_t kNegInfBits = 0xff800000u;
-constexpr int REG_LO = 56, REG_HI = 216; // 128 * 56 + 256 * 216 = 62464 <= 384 * 168
+constexpr int REG_LAUNCH = 128; // 65536 registers / 512 threads
+constexpr int REG_PRODUCER = 56, REG_SOFTMAX = 184, REG_EPILOGUE = 88;
+static_assert(REG_PRODUCER + 2 * REG_SOFTMAX + REG_EPILOGUE <= 4 * REG_LAUNCH, "register split exceeds the launch budget");
+
+__device__ __forceinline__ uint32_t a_col(int t) { return (uint32_t)(t & 1) * 128; }
+__device__ __forceinline__ uint32_t o_col(int t) { return 256u + (uint32_t)(t & 1) * 128; }
 
 template <int DH, int G>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     sparse_attn_kernel(AttnArgs a, const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap)
 {
@@ -65,6 +82,7 @@ __global__ void __launch_bounds__(384, 1)
     AttnShared& sh = *reinterpret_cast<AttnShared*>(sV + 2 * C::TILE);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wg = warp >> 2;
     const int P = gridDim.x, cta = blockIdx.x;
     const int64_t Nk = a.N * a.k;
     volatile int* abort_flag = &sh.abort_flag;
@@ -73,15 +91,18 @@ __global__ void __launch_bounds__(384, 1)
     const bool tl_on = a.timeline != nullptr && cta == 0;
 #define TL(slot, tile)                                                                                    \
     do {                                                                                                  \
-        if (tl_on && (tile) < a.timeline_tiles) a.timeline[(int64_t)(tile) * 10 + (slot)] = clock64();    \
+        if (tl_on && (tile) < a.timeline_tiles) a.timeline[(int64_t)(tile) * 16 + (slot)] = clock64();    \
     } while (0)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh.kv_full[i], 1);
             mbar_init(&sh.kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&sh.s_full[i], 1);
             mbar_init(&sh.p_full[i], 4);
+            mbar_init(&sh.pv_done[i], 1);
             mbar_init(&sh.o_full[i], 1);
             mbar_init(&sh.o_free[i], 4);
         }
@@ -89,7 +110,9 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&sh.q_full[i], 1);
             mbar_init(&sh.q_empty[i], 1);
         }
+        for (int i = 0; i < 4; ++i) mbar_init(&sh.ml_full[i], 4);
         mbar_init(&sh.done, 1);
+        mbar_init(&sh.done2, 1);
         sh.abort_flag = 0;
         fence_mbar_init();
     }
@@ -102,146 +125,162 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
 
-    // Register split (each warpgroup executes its own setmaxnreg inside its branch): 384 threads x
-    // 168 launch registers = 64512 >= producer warpgroup 128 x REG_LO + softmax warpgroups 256 x REG_HI.
-    if (warp < 4) {
-        reg_dealloc<REG_LO>();
-    if (warp == 0) {
-        // ------------------------------------------------------------ K/V producer
-        if (lane == 0) {
-            int it = 0;
-            for (int j = j_begin; j < j_end; j += P, ++it) {
-                const msa_work_item item = a.items[j];
-                const int s = it & 1;
-                if (!wait_or_abort(&sh.kv_empty[s], ((it >> 1) & 1) ^ 1, abort_flag, a.err, 20, kWaitLimit)) break;
-                mbar_arrive_expect_tx(&sh.kv_full[s], 2 * C::TILE);
-                for (int c = 0; c < C::NKC; ++c) {
-                    tma_load_3d(sK + s * C::TILE + c * C::CHUNK, &kmap, &sh.kv_full[s], c * 64, item.r, item.b * kBk);
-                    tma_load_3d(sV + s * C::TILE + c * C::CHUNK, &vmap, &sh.kv_full[s], c * 64, item.r, item.b * kBk);
-                }
-            }
-            for (int g = it - 1; g >= 0 && g >= it - 2; --g) mbar_wait(&sh.kv_full[g & 1], (g >> 1) & 1, kWaitLimit);
-        }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------ Q gather (TMA per position)
-        int qt = 0;
-        bool ok = true;
-        for (int j = j_begin; j < j_end && ok; j += P) {
-            const msa_work_item item = a.items[j];
-            const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
-            const int ntiles = (item.len + PPT - 1) / PPT;
-            for (int t = 0; t < ntiles; ++t, ++qt) {
-                const int qs = qt % NQ;
-                const int npos = min(PPT, item.len - t * PPT);
-                // fetch this tile's rows before waiting for the stage
-                int prow[(PPT + 31) / 32];
-#pragma unroll
-                for (int u = 0; u < (PPT + 31) / 32; ++u) {
-                    const int pl = lane + 32 * u;
-                    prow[u] = pl < npos ? ent[t * PPT + pl] / a.k : 0;
-                }
-                int w_ok = 1;
-                if (lane == 0)
-                    w_ok = wait_or_abort(&sh.q_empty[qs], ((qt / NQ) & 1) ^ 1, abort_flag, a.err, 21, kWaitLimit);
-                w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-                if (!w_ok) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
-                    TL(0, qt);
-                    mbar_arrive_expect_tx(&sh.q_full[qs], npos * G * DH * 2);
-                }
-                __syncwarp();
-#pragma unroll
-                for (int u = 0; u < (PPT + 31) / 32; ++u) {
-                    const int pl = lane + 32 * u;
-                    if (pl < npos) {
-#pragma unroll
-                        for (int c = 0; c < C::NKC; ++c)
-                            tma_load_3d(sQ + qs * C::TILE + c * C::CHUNK + pl * G * 128, &qmap, &sh.q_full[qs], c * 64,
-                                        item.r * G, prow[u]);
+    if (wg == 0) {
+        reg_set<REG_PRODUCER, REG_LAUNCH>();
+        if (warp == 0) {
+            // -------------------------------------------------------- K/V producer
+            if (lane == 0) {
+                int it = 0;
+                for (int j = j_begin; j < j_end; j += P, ++it) {
+                    const msa_work_item item = a.items[j];
+                    const int s = it & 1;
+                    if (!wait_or_abort(&sh.kv_empty[s], ((it >> 1) & 1) ^ 1, abort_flag, a.err, 20, kWaitLimit))
+                        break;
+                    mbar_arrive_expect_tx(&sh.kv_full[s], 2 * C::TILE);
+                    for (int c = 0; c < C::NKC; ++c) {
+                        tma_load_3d(sK + s * C::TILE + c * C::CHUNK, &kmap, &sh.kv_full[s], c * 64, item.r,
+                                    item.b * kBk);
+                        tma_load_3d(sV + s * C::TILE + c * C::CHUNK, &vmap, &sh.kv_full[s], c * 64, item.r,
+                                    item.b * kBk);
                     }
                 }
-                if (lane == 0) TL(1, qt);
+                for (int g = it - 1; g >= 0 && g >= it - 2; --g)
+                    mbar_wait(&sh.kv_full[g & 1], (g >> 1) & 1, kWaitLimit);
             }
-        }
-        if (lane == 0)
-            for (int g = qt - 1; g >= 0 && g >= qt - NQ; --g) mbar_wait(&sh.q_full[g % NQ], (g / NQ) & 1, kWaitLimit);
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
-            constexpr uint32_t idPV = idesc_bf16_f32(128, DH, true);
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-            int qt = 0, it = 0;
-            int prev_qt = -1, prev_kvs = 0;
-            bool prev_last = false, ok = true;
-            // O(pqt) = P(pqt) V: needs P written and the O buffer read by the epilogue of pqt-2
-            auto issue_pv = [&](int pqt, int pkvs, bool plast) -> bool {
-                const int pb = pqt & 1;
-                if (!wait_or_abort(&sh.p_full[pb], (pqt >> 1) & 1, abort_flag, a.err, 22, kWaitLimit)) return false;
-                if (!wait_or_abort(&sh.o_free[pb], ((pqt >> 1) & 1) ^ 1, abort_flag, a.err, 28, kWaitLimit))
-                    return false;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_ts(tmem + 256 + pb * 128, tmem + pb * 128 + ks * 8,
-                           smem_desc(aV + pkvs * C::TILE + ks * 2048, C::CHUNK, 1024, 128), idPV, ks > 0);
-                tc_commit(&sh.o_full[pb]);
-                if (plast) tc_commit(&sh.kv_empty[pkvs]);
-                TL(3, pqt);
-                return true;
-            };
-            for (int j = j_begin; j < j_end && ok; j += P, ++it) {
+        } else if (warp == 2) {
+            // -------------------------------------------------------- Q gather (TMA per position)
+            int qt = 0;
+            bool ok = true;
+            for (int j = j_begin; j < j_end && ok; j += P) {
                 const msa_work_item item = a.items[j];
-                const int kvs = it & 1;
+                const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
                 const int ntiles = (item.len + PPT - 1) / PPT;
-                if (!wait_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 23, kWaitLimit)) break;
-                TL(8, qt);
                 for (int t = 0; t < ntiles; ++t, ++qt) {
-                    const int buf = qt & 1, qs = qt % NQ;
-                    // S/P buffer is free once PV(qt-2) has completed
-                    if (!wait_or_abort(&sh.q_full[qs], (qt / NQ) & 1, abort_flag, a.err, 24, kWaitLimit) ||
-                        (qt >= 2 && !wait_or_abort(&sh.o_full[buf], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 25,
-                                                   kWaitLimit))) {
-                        ok = false;
-                        break;
-                    }
-                    TL(9, qt);
-                    tc_fence_after();
+                    const int qs = qt % NQ;
+                    const int npos = min(PPT, item.len - t * PPT);
+                    // fetch this tile's rows before waiting for the stage
+                    int prow[(PPT + 31) / 32];
 #pragma unroll
-                    for (int ks = 0; ks < DH / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * C::CHUNK + (ks & 3) * 32;
-                        mma_ss(tmem + buf * 128, desc_kmajor(aQ + qs * C::TILE + off, 128),
-                               desc_kmajor(aK + kvs * C::TILE + off, 128), idS, ks > 0);
+                    for (int u = 0; u < (PPT + 31) / 32; ++u) {
+                        const int pl = lane + 32 * u;
+                        prow[u] = pl < npos ? ent[t * PPT + pl] / a.k : 0;
                     }
-                    tc_commit(&sh.s_full[buf]);
-                    tc_commit(&sh.q_empty[qs]);
-                    TL(2, qt);
-                    if (prev_qt >= 0 && !issue_pv(prev_qt, prev_kvs, prev_last)) {
+                    int w_ok = 1;
+                    if (lane == 0)
+                        w_ok = wait_or_abort(&sh.q_empty[qs], ((qt / NQ) & 1) ^ 1, abort_flag, a.err, 21, kWaitLimit);
+                    w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+                    if (!w_ok) {
                         ok = false;
                         break;
                     }
-                    prev_qt = qt;
-                    prev_kvs = kvs;
-                    prev_last = (t == ntiles - 1);
+                    if (lane == 0) {
+                        TL(0, qt);
+                        mbar_arrive_expect_tx(&sh.q_full[qs], npos * G * DH * 2);
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int u = 0; u < (PPT + 31) / 32; ++u) {
+                        const int pl = lane + 32 * u;
+                        if (pl < npos) {
+#pragma unroll
+                            for (int c = 0; c < C::NKC; ++c)
+                                tma_load_3d(sQ + qs * C::TILE + c * C::CHUNK + pl * G * 128, &qmap, &sh.q_full[qs],
+                                            c * 64, item.r * G, prow[u]);
+                        }
+                    }
+                    if (lane == 0) TL(1, qt);
                 }
             }
-            if (ok && prev_qt >= 0) issue_pv(prev_qt, prev_kvs, prev_last);
-            tc_commit(&sh.done);
-            mbar_wait(&sh.done, 0, kWaitLimit);
+            if (lane == 0)
+                for (int g = qt - 1; g >= 0 && g >= qt - NQ; --g)
+                    mbar_wait(&sh.q_full[g % NQ], (g / NQ) & 1, kWaitLimit);
+        } else if (warp == 1) {
+            // -------------------------------------------------------- S issuer: S(t) = Q K^T
+            if (lane == 0) {
+                constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
+                const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
+                int qt = 0, it = 0;
+                bool ok = true;
+                for (int j = j_begin; j < j_end && ok; j += P, ++it) {
+                    const msa_work_item item = a.items[j];
+                    const int kvs = it & 1;
+                    const int ntiles = (item.len + PPT - 1) / PPT;
+                    if (!poll_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 23, kWaitLimit)) break;
+                    TL(8, qt);
+                    const uint64_t kdesc = desc_kmajor(aK + kvs * C::TILE, 128);
+                    for (int t = 0; t < ntiles; ++t, ++qt) {
+                        const int qa = qt & 1, qs = qt % NQ;
+                        // A[qt % 2] is free once PV(qt-2) has consumed P(qt-2)
+                        if (!poll_or_abort(&sh.q_full[qs], (qt / NQ) & 1, abort_flag, a.err, 24, kWaitLimit) ||
+                            (qt >= 2 && !poll_or_abort(&sh.pv_done[qa], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 25,
+                                                       kWaitLimit))) {
+                            ok = false;
+                            break;
+                        }
+                        TL(9, qt);
+                        tc_fence_after();
+                        const uint64_t qdesc = desc_kmajor(aQ + qs * C::TILE, 128);
+                        const uint32_t sd = tmem + a_col(qt);
+#pragma unroll
+                        for (int ks = 0; ks < DH / 16; ++ks) {
+                            const uint64_t off = (uint64_t)((((ks >> 2) * C::CHUNK) + (ks & 3) * 32) >> 4);
+                            mma_ss(sd, qdesc + off, kdesc + off, idS, ks > 0);
+                        }
+                        tc_commit(&sh.s_full[qa]);
+                        tc_commit(&sh.q_empty[qs]);
+                        TL(2, qt);
+                    }
+                }
+                tc_commit(&sh.done);
+                mbar_wait(&sh.done, 0, kWaitLimit);
+            }
+        } else if (warp == 3) {
+            // -------------------------------------------------------- PV issuer: O(t) = P(t) V
+            if (lane == 0) {
+                constexpr uint32_t idPV = idesc_bf16_f32(128, DH, true);
+                const uint32_t aV = smem_u32(sV);
+                int qt = 0, it = 0;
+                bool ok = true;
+                for (int j = j_begin; j < j_end && ok; j += P, ++it) {
+                    const msa_work_item item = a.items[j];
+                    const int kvs = it & 1;
+                    const int ntiles = (item.len + PPT - 1) / PPT;
+                    if (!poll_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 30, kWaitLimit)) break;
+                    const uint64_t vdesc = smem_desc(aV + kvs * C::TILE, C::CHUNK, 1024, 128);
+                    for (int t = 0; t < ntiles; ++t, ++qt) {
+                        const int pa = qt & 1;
+                        TL(10, qt);
+                        // needs P(qt) and the epilogue of qt-2 to have read O[qt % 2]
+                        if (!poll_or_abort(&sh.p_full[pa], (qt >> 1) & 1, abort_flag, a.err, 22, kWaitLimit) ||
+                            (qt >= 2 && !poll_or_abort(&sh.o_free[pa], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 28,
+                                                       kWaitLimit))) {
+                            ok = false;
+                            break;
+                        }
+                        TL(12, qt);
+                        tc_fence_after();
+                        const uint32_t acol = tmem + a_col(qt);
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks) // 16 keys = 2048 bytes of V per step
+                            mma_ts(tmem + o_col(qt), acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
+                        tc_commit(&sh.pv_done[pa]);
+                        tc_commit(&sh.o_full[pa]);
+                        if (t == ntiles - 1) tc_commit(&sh.kv_empty[kvs]);
+                        TL(3, qt);
+                    }
+                }
+                tc_commit(&sh.done2);
+                mbar_wait(&sh.done2, 0, kWaitLimit);
+            }
         }
-    }
-    } else {
-        reg_alloc<REG_HI>();
-        // ------------------------------------------------------------ softmax + epilogue
-        const int beta = (warp - 4) >> 2;
+    } else if (wg <= 2) {
+        reg_set<REG_SOFTMAX, REG_LAUNCH>();
+        // ------------------------------------------------------------ softmax
+        const int beta = wg - 1;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const int pl = row / G, hh = row % G;
-        const float scale = rsqrtf((float)DH);
-        const float sl2 = scale * 1.4426950408889634f;
+        const int pl = row / G;
+        const float sl2 = rsqrtf((float)DH) * 1.4426950408889634f;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         int qt = 0;
         bool ok = true;
@@ -251,32 +290,28 @@ __global__ void __launch_bounds__(384, 1)
             const int ntiles = (item.len + PPT - 1) / PPT;
             for (int t = 0; t < ntiles; ++t, ++qt) {
                 if ((qt & 1) != beta) continue;
-                const int buf = beta;
+                const int qa = qt & 1;
                 const int idx = t * PPT + pl;
-                const bool valid = idx < item.len;
-                const int32_t e = valid ? ent[idx] : 0;
-                const int p = e / a.k;
-                const int slot = e - p * a.k;
-                const int limit = valid ? min(127, p - item.b * kBk) : 127;
-                if (!wait_or_abort(&sh.s_full[buf], (qt >> 1) & 1, abort_flag, a.err, 26, kWaitLimit)) {
+                const int limit = idx < item.len ? min(127, ent[idx] / a.k - item.b * kBk) : 127;
+                if (!wait_or_abort(&sh.s_full[qa], (qt >> 1) & 1, abort_flag, a.err, 26, kWaitLimit)) {
                     ok = false;
                     break;
                 }
                 if (row == 0) TL(4, qt);
                 tc_fence_after();
-                const uint32_t sadr = lane_base + buf * 128;
+                const uint32_t sadr = lane_base + a_col(qt);
                 uint32_t s[128];
                 tmem_ld32_at<0>(sadr, s);
                 tmem_ld32_at<32>(sadr + 32, s);
                 tmem_ld32_at<64>(sadr + 64, s);
                 tmem_ld32_at<96>(sadr + 96, s);
                 tmem_ld_wait();
+                if (row == 0) TL(14, qt);
                 if (limit < 127) { // the query's own block: keys after the query are invisible
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
                         if (c > limit) s[c] = kNegInfBits;
                 }
-                // row max: 3-input max tree
                 float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F;
 #pragma unroll
                 for (int c = 0; c < 128; c += 4) {
@@ -301,33 +336,47 @@ __global__ void __launch_bounds__(384, 1)
                     }
                     tmem_st16(sadr + c4 * 16, pk);
                 }
+                sh.ml[qt & 3][row] = make_float2(m, f2_lo(l2) + f2_hi(l2));
                 tmem_st_wait();
-                const float l = f2_lo(l2) + f2_hi(l2);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.p_full[buf]);
+                if (lane == 0) {
+                    mbar_arrive(&sh.p_full[qa]);
+                    mbar_arrive(&sh.ml_full[qt & 3]);
+                }
                 if (row == 0) TL(5, qt);
-
-                // epilogue: O / l -> partial slot, lse
-                if (!wait_or_abort(&sh.o_full[buf], (qt >> 1) & 1, abort_flag, a.err, 27, kWaitLimit)) {
+            }
+        }
+    } else {
+        reg_set<REG_EPILOGUE, REG_LAUNCH>();
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int pl = row / G, hh = row % G;
+        const float scale = rsqrtf((float)DH);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        int qt = 0;
+        bool ok = true;
+        for (int j = j_begin; j < j_end && ok; j += P) {
+            const msa_work_item item = a.items[j];
+            const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
+            const int ntiles = (item.len + PPT - 1) / PPT;
+            for (int t = 0; t < ntiles; ++t, ++qt) {
+                if (row == 0) TL(15, qt);
+                const int idx = t * PPT + pl;
+                const bool valid = idx < item.len;
+                const int32_t e = valid ? ent[idx] : 0;
+                const int p = e / a.k;
+                const int slot = e - p * a.k;
+                if (!wait_or_abort(&sh.o_full[qt & 1], (qt >> 1) & 1, abort_flag, a.err, 27, kWaitLimit) ||
+                    !wait_or_abort(&sh.ml_full[qt & 3], (qt >> 2) & 1, abort_flag, a.err, 29, kWaitLimit)) {
                     ok = false;
                     break;
                 }
                 if (row == 0) TL(6, qt);
                 tc_fence_after();
-                const uint32_t oadr = lane_base + 256 + buf * 128;
-                uint32_t o[DH];
-                tmem_ld32_at<0>(oadr, o);
-                tmem_ld32_at<32>(oadr + 32, o);
-                if constexpr (DH == 128) {
-                    tmem_ld32_at<64 % DH>(oadr + 64, o);
-                    tmem_ld32_at<96 % DH>(oadr + 96, o);
-                }
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.o_free[buf]);
-                const float inv_l = 1.f / l;
+                const float2 ml = sh.ml[qt & 3][row];
+                const float inv_l = 1.f / ml.y;
                 const int h = item.r * G + hh;
                 const int64_t prow = (int64_t)(p - a.row0);
                 bool store = valid;
@@ -335,25 +384,37 @@ __global__ void __launch_bounds__(384, 1)
                     report_error(a.err, MSA_ERR_DEVICE_CHECK, 300); // entry outside this pass: skip it
                     store = false;
                 }
-                if (store) {
-                    // partial layout [row][slot][d_h/8][H_q][8]: the G heads of a position are adjacent
-                    // 16-byte units, so each warp-wide store writes contiguous runs
-                    uint4* d4 = reinterpret_cast<uint4*>(a.o_part + (prow * a.k + slot) * (int64_t)a.H_q * DH) + h;
-                    const uint64_t il2 = f2_pack(inv_l, inv_l);
+                // partial layout [row][slot][d_h/8][H_q][8]: the G heads of a position are adjacent
+                // 16-byte units, so each warp-wide store writes contiguous runs
+                uint4* d4 = reinterpret_cast<uint4*>(a.o_part + (prow * a.k + slot) * (int64_t)a.H_q * DH) + h;
+                const uint64_t il2 = f2_pack(inv_l, inv_l);
 #pragma unroll
-                    for (int q = 0; q < DH / 8; ++q) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int z = 0; z < 4; ++z) {
-                            const uint64_t y = f2_mul(f2_pack(__uint_as_float(o[8 * q + 2 * z]),
-                                                              __uint_as_float(o[8 * q + 2 * z + 1])),
-                                                      il2);
-                            w[z] = pack_bf16x2(f2_lo(y), f2_hi(y));
-                        }
-                        d4[q * a.H_q] = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int c = 0; c < DH / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(lane_base + o_col(qt) + c * 32, o);
+                    tmem_ld_wait();
+                    if (c == DH / 32 - 1) { // O fully read: PV of the next tile may overwrite it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sh.o_free[qt & 1]);
+                        if (row == 0) TL(13, qt);
                     }
-                    a.lse_part[(prow * a.k + slot) * a.H_q + h] = m * scale + logf(l);
+                    if (store) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int z = 0; z < 4; ++z) {
+                                const uint64_t y = f2_mul(
+                                    f2_pack(__uint_as_float(o[8 * q + 2 * z]), __uint_as_float(o[8 * q + 2 * z + 1])),
+                                    il2);
+                                w[z] = pack_bf16x2(f2_lo(y), f2_hi(y));
+                            }
+                            d4[(c * 4 + q) * a.H_q] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
                 }
+                if (store) a.lse_part[(prow * a.k + slot) * a.H_q + h] = ml.x * scale + logf(ml.y);
                 if (row == 0) TL(7, qt);
             }
         }
@@ -362,8 +423,8 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, 512);
-}
 #undef TL
+}
 
 template <int DH, int G>
 cudaError_t launch_cfg(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
@@ -374,7 +435,7 @@ cudaError_t launch_cfg(const AttnArgs& a, const CUtensorMap& qmap, const CUtenso
     static_assert(AttnCfg<DH>::SMEM + sizeof(AttnShared) <= 227 * 1024, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    sparse_attn_kernel<DH, G><<<n_sm, 384, smem, s>>>(a, qmap, kmap, vmap);
+    sparse_attn_kernel<DH, G><<<n_sm, 512, smem, s>>>(a, qmap, kmap, vmap);
     note_launch(1);
     return cudaGetLastError();
 }
