@@ -15,8 +15,12 @@
 // (combine.cu) merges the <= k partials of every (row, head) through their lse.
 //
 // Roles (512 threads, four warpgroups):
-//   WG0: warp 0 = K/V TMA producer, warp 1 = S issuer + TMEM owner, warp 2 = Q gather (one TMA
-//        box per position, issued by the 32 lanes in parallel), warp 3 = PV issuer
+//   WG0: warp 0 = K/V TMA producer, warp 1 = S issuer + TMEM owner, warp 2 = tile scheduler and Q
+//        gather (one TMA box per position, issued by the 32 lanes in parallel), warp 3 = PV issuer
+// The tile scheduler is the only role that reads the work list in global memory after the K/V
+// producer: it publishes every tile as a record (group, block, positions, their entries, item
+// boundaries) in a shared-memory ring that the MMA issuers, the softmax and the epilogue consume,
+// so none of them waits on a global load. The epilogue releases a record after its tile's PV.
 //   WG1, WG2: softmax of even / odd tiles
 //   WG3: epilogue of every tile (O / rowsum -> partial slot)
 // TMEM (512 columns): two 128-column S/P regions A[t % 2] at columns 0 and 128 (S, then P in
@@ -46,14 +50,25 @@ struct AttnCfg {
     static constexpr int SMEM = 1024 + NQ * TILE + 4 * TILE;
 };
 
+constexpr int kRing = 8; // tile records in flight between the scheduler and the epilogue
+
+struct TileRec {
+    int32_t r, b;  // GQA group, KV block
+    int32_t npos;  // positions in the tile (1 .. 128/G); -1 marks the end of the CTA's work
+    int32_t flags; // bit 0: first tile of its item, bit 1: last tile, bit 2: K/V stage of the item
+};
+
 struct AttnShared {
     uint64_t kv_full[2], kv_empty[2];
     uint64_t q_full[2], q_empty[2];
     uint64_t s_full[2], p_full[2], pv_done[2];
     uint64_t o_full[2], o_free[2];
     uint64_t ml_full[4];
+    uint64_t tile_full[kRing], tile_free[kRing];
     uint64_t done, done2;
     float2 ml[4][128]; // (row max of the raw scores, row sum of exp) per tile slot and row
+    TileRec rec[kRing];
+    int32_t rec_e[kRing][128]; // entry (i*k + slot) of each position of the tile
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -111,6 +126,10 @@ __global__ void __launch_bounds__(512, 1)
             mbar_init(&sh.q_empty[i], 1);
         }
         for (int i = 0; i < 4; ++i) mbar_init(&sh.ml_full[i], 4);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(&sh.tile_full[i], 1);
+            mbar_init(&sh.tile_free[i], 4);
+        }
         mbar_init(&sh.done, 1);
         mbar_init(&sh.done2, 1);
         sh.abort_flag = 0;
@@ -148,24 +167,50 @@ __global__ void __launch_bounds__(512, 1)
                     mbar_wait(&sh.kv_full[g & 1], (g >> 1) & 1, kWaitLimit);
             }
         } else if (warp == 2) {
-            // -------------------------------------------------------- Q gather (TMA per position)
-            int qt = 0;
+            // -------------------------------------------------------- tile scheduler + Q gather
+            int qt = 0, it = 0;
             bool ok = true;
-            for (int j = j_begin; j < j_end && ok; j += P) {
+            for (int j = j_begin; j < j_end && ok; j += P, ++it) {
                 const msa_work_item item = a.items[j];
+                if (item.len <= 0) { // the inversion never emits empty items; stop rather than desynchronise
+                    if (lane == 0) {
+                        report_error(a.err, MSA_ERR_DEVICE_CHECK, 301);
+                        *abort_flag = 1;
+                    }
+                    ok = false;
+                    break;
+                }
                 const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
                 const int ntiles = (item.len + PPT - 1) / PPT;
                 for (int t = 0; t < ntiles; ++t, ++qt) {
-                    const int qs = qt % NQ;
+                    const int qs = qt % NQ, rs = qt % kRing;
                     const int npos = min(PPT, item.len - t * PPT);
-                    // fetch this tile's rows before waiting for the stage
-                    int prow[(PPT + 31) / 32];
+                    // fetch this tile's entries before waiting for anything
+                    int e[(PPT + 31) / 32];
 #pragma unroll
                     for (int u = 0; u < (PPT + 31) / 32; ++u) {
                         const int pl = lane + 32 * u;
-                        prow[u] = pl < npos ? ent[t * PPT + pl] / a.k : 0;
+                        e[u] = pl < npos ? ent[t * PPT + pl] : 0;
                     }
                     int w_ok = 1;
+                    if (lane == 0 && qt >= kRing)
+                        w_ok = wait_or_abort(&sh.tile_free[rs], ((qt / kRing) & 1) ^ 1, abort_flag, a.err, 33,
+                                             kWaitLimit);
+                    w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+                    if (!w_ok) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int u = 0; u < (PPT + 31) / 32; ++u) {
+                        const int pl = lane + 32 * u;
+                        if (pl < npos) sh.rec_e[rs][pl] = e[u];
+                    }
+                    if (lane == 0)
+                        sh.rec[rs] = TileRec{item.r, item.b, npos,
+                                             (t == 0 ? 1 : 0) | (t == ntiles - 1 ? 2 : 0) | ((it & 1) << 2)};
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sh.tile_full[rs]);
                     if (lane == 0)
                         w_ok = wait_or_abort(&sh.q_empty[qs], ((qt / NQ) & 1) ^ 1, abort_flag, a.err, 21, kWaitLimit);
                     w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
@@ -185,51 +230,64 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
                             for (int c = 0; c < C::NKC; ++c)
                                 tma_load_3d(sQ + qs * C::TILE + c * C::CHUNK + pl * G * 128, &qmap, &sh.q_full[qs],
-                                            c * 64, item.r * G, prow[u]);
+                                            c * 64, item.r * G, e[u] / a.k);
                         }
                     }
                     if (lane == 0) TL(1, qt);
                 }
             }
+            const int n_tiles = qt;
+            // two end records, so that each softmax warpgroup (even / odd tiles) meets one
+            if (lane == 0 && ok) {
+                for (int z = 0; z < 2; ++z, ++qt) {
+                    const int rs = qt % kRing;
+                    if (qt >= kRing && !wait_or_abort(&sh.tile_free[rs], ((qt / kRing) & 1) ^ 1, abort_flag, a.err,
+                                                      33, kWaitLimit))
+                        break;
+                    sh.rec[rs] = TileRec{0, 0, -1, 0};
+                    mbar_arrive(&sh.tile_full[rs]);
+                }
+            }
             if (lane == 0)
-                for (int g = qt - 1; g >= 0 && g >= qt - NQ; --g)
+                for (int g = n_tiles - 1; g >= 0 && g >= n_tiles - NQ; --g)
                     mbar_wait(&sh.q_full[g % NQ], (g / NQ) & 1, kWaitLimit);
         } else if (warp == 1) {
             // -------------------------------------------------------- S issuer: S(t) = Q K^T
             if (lane == 0) {
                 constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
                 const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
-                int qt = 0, it = 0;
-                bool ok = true;
-                for (int j = j_begin; j < j_end && ok; j += P, ++it) {
-                    const msa_work_item item = a.items[j];
-                    const int kvs = it & 1;
-                    const int ntiles = (item.len + PPT - 1) / PPT;
-                    if (!poll_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 23, kWaitLimit)) break;
-                    TL(8, qt);
-                    const uint64_t kdesc = desc_kmajor(aK + kvs * C::TILE, 128);
-                    for (int t = 0; t < ntiles; ++t, ++qt) {
-                        const int qa = qt & 1, qs = qt % NQ;
-                        // A[qt % 2] is free once PV(qt-2) has consumed P(qt-2)
-                        if (!poll_or_abort(&sh.q_full[qs], (qt / NQ) & 1, abort_flag, a.err, 24, kWaitLimit) ||
-                            (qt >= 2 && !poll_or_abort(&sh.pv_done[qa], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 25,
-                                                       kWaitLimit))) {
-                            ok = false;
-                            break;
-                        }
-                        TL(9, qt);
-                        tc_fence_after();
-                        const uint64_t qdesc = desc_kmajor(aQ + qs * C::TILE, 128);
-                        const uint32_t sd = tmem + a_col(qt);
-#pragma unroll
-                        for (int ks = 0; ks < DH / 16; ++ks) {
-                            const uint64_t off = (uint64_t)((((ks >> 2) * C::CHUNK) + (ks & 3) * 32) >> 4);
-                            mma_ss(sd, qdesc + off, kdesc + off, idS, ks > 0);
-                        }
-                        tc_commit(&sh.s_full[qa]);
-                        tc_commit(&sh.q_empty[qs]);
-                        TL(2, qt);
+                int it = -1;
+                uint64_t kdesc = 0;
+                for (int qt = 0;; ++qt) {
+                    const int rs = qt % kRing;
+                    if (!poll_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 34, kWaitLimit)) break;
+                    const TileRec rec = sh.rec[rs];
+                    if (rec.npos < 0) break;
+                    const int kvs = (rec.flags >> 2) & 1;
+                    if (rec.flags & 1) {
+                        ++it;
+                        if (!poll_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 23, kWaitLimit)) break;
+                        TL(8, qt);
+                        kdesc = desc_kmajor(aK + kvs * C::TILE, 128);
                     }
+                    const int qa = qt & 1, qs = qt % NQ;
+                    // A[qt % 2] is free once PV(qt-2) has consumed P(qt-2)
+                    if (!poll_or_abort(&sh.q_full[qs], (qt / NQ) & 1, abort_flag, a.err, 24, kWaitLimit) ||
+                        (qt >= 2 && !poll_or_abort(&sh.pv_done[qa], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 25,
+                                                   kWaitLimit)))
+                        break;
+                    TL(9, qt);
+                    tc_fence_after();
+                    const uint64_t qdesc = desc_kmajor(aQ + qs * C::TILE, 128);
+                    const uint32_t sd = tmem + a_col(qt);
+#pragma unroll
+                    for (int ks = 0; ks < DH / 16; ++ks) {
+                        const uint64_t off = (uint64_t)((((ks >> 2) * C::CHUNK) + (ks & 3) * 32) >> 4);
+                        mma_ss(sd, qdesc + off, kdesc + off, idS, ks > 0);
+                    }
+                    tc_commit(&sh.s_full[qa]);
+                    tc_commit(&sh.q_empty[qs]);
+                    TL(2, qt);
                 }
                 tc_commit(&sh.done);
                 mbar_wait(&sh.done, 0, kWaitLimit);
@@ -239,35 +297,36 @@ __global__ void __launch_bounds__(512, 1)
             if (lane == 0) {
                 constexpr uint32_t idPV = idesc_bf16_f32(128, DH, true);
                 const uint32_t aV = smem_u32(sV);
-                int qt = 0, it = 0;
-                bool ok = true;
-                for (int j = j_begin; j < j_end && ok; j += P, ++it) {
-                    const msa_work_item item = a.items[j];
-                    const int kvs = it & 1;
-                    const int ntiles = (item.len + PPT - 1) / PPT;
-                    if (!poll_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 30, kWaitLimit)) break;
-                    const uint64_t vdesc = smem_desc(aV + kvs * C::TILE, C::CHUNK, 1024, 128);
-                    for (int t = 0; t < ntiles; ++t, ++qt) {
-                        const int pa = qt & 1;
-                        TL(10, qt);
-                        // needs P(qt) and the epilogue of qt-2 to have read O[qt % 2]
-                        if (!poll_or_abort(&sh.p_full[pa], (qt >> 1) & 1, abort_flag, a.err, 22, kWaitLimit) ||
-                            (qt >= 2 && !poll_or_abort(&sh.o_free[pa], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 28,
-                                                       kWaitLimit))) {
-                            ok = false;
-                            break;
-                        }
-                        TL(12, qt);
-                        tc_fence_after();
-                        const uint32_t acol = tmem + a_col(qt);
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) // 16 keys = 2048 bytes of V per step
-                            mma_ts(tmem + o_col(qt), acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
-                        tc_commit(&sh.pv_done[pa]);
-                        tc_commit(&sh.o_full[pa]);
-                        if (t == ntiles - 1) tc_commit(&sh.kv_empty[kvs]);
-                        TL(3, qt);
+                int it = -1;
+                uint64_t vdesc = 0;
+                for (int qt = 0;; ++qt) {
+                    const int rs = qt % kRing;
+                    if (!poll_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 35, kWaitLimit)) break;
+                    const TileRec rec = sh.rec[rs];
+                    if (rec.npos < 0) break;
+                    const int kvs = (rec.flags >> 2) & 1;
+                    if (rec.flags & 1) {
+                        ++it;
+                        if (!poll_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 30, kWaitLimit)) break;
+                        vdesc = smem_desc(aV + kvs * C::TILE, C::CHUNK, 1024, 128);
                     }
+                    const int pa = qt & 1;
+                    TL(10, qt);
+                    // needs P(qt) and the epilogue of qt-2 to have read O[qt % 2]
+                    if (!poll_or_abort(&sh.p_full[pa], (qt >> 1) & 1, abort_flag, a.err, 22, kWaitLimit) ||
+                        (qt >= 2 && !poll_or_abort(&sh.o_free[pa], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 28,
+                                                   kWaitLimit)))
+                        break;
+                    TL(12, qt);
+                    tc_fence_after();
+                    const uint32_t acol = tmem + a_col(qt);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) // 16 keys = 2048 bytes of V per step
+                        mma_ts(tmem + o_col(qt), acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
+                    tc_commit(&sh.pv_done[pa]);
+                    tc_commit(&sh.o_full[pa]);
+                    if (rec.flags & 2) tc_commit(&sh.kv_empty[kvs]);
+                    TL(3, qt);
                 }
                 tc_commit(&sh.done2);
                 mbar_wait(&sh.done2, 0, kWaitLimit);
@@ -282,70 +341,62 @@ __global__ void __launch_bounds__(512, 1)
         const int pl = row / G;
         const float sl2 = rsqrtf((float)DH) * 1.4426950408889634f;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        int qt = 0;
-        bool ok = true;
-        for (int j = j_begin; j < j_end && ok; j += P) {
-            const msa_work_item item = a.items[j];
-            const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
-            const int ntiles = (item.len + PPT - 1) / PPT;
-            for (int t = 0; t < ntiles; ++t, ++qt) {
-                if ((qt & 1) != beta) continue;
-                const int qa = qt & 1;
-                const int idx = t * PPT + pl;
-                const int limit = idx < item.len ? min(127, ent[idx] / a.k - item.b * kBk) : 127;
-                if (!wait_or_abort(&sh.s_full[qa], (qt >> 1) & 1, abort_flag, a.err, 26, kWaitLimit)) {
-                    ok = false;
-                    break;
-                }
-                if (row == 0) TL(4, qt);
-                tc_fence_after();
-                const uint32_t sadr = lane_base + a_col(qt);
-                uint32_t s[128];
-                tmem_ld32_at<0>(sadr, s);
-                tmem_ld32_at<32>(sadr + 32, s);
-                tmem_ld32_at<64>(sadr + 64, s);
-                tmem_ld32_at<96>(sadr + 96, s);
-                tmem_ld_wait();
-                if (row == 0) TL(14, qt);
-                if (limit < 127) { // the query's own block: keys after the query are invisible
+        for (int qt = beta;; qt += 2) {
+            const int rs = qt % kRing;
+            if (!wait_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 36, kWaitLimit)) break;
+            const TileRec rec = sh.rec[rs];
+            if (rec.npos < 0) break;
+            const int qa = qt & 1;
+            const int limit = pl < rec.npos ? min(127, sh.rec_e[rs][pl] / a.k - rec.b * kBk) : 127;
+            if (!wait_or_abort(&sh.s_full[qa], (qt >> 1) & 1, abort_flag, a.err, 26, kWaitLimit)) break;
+            if (row == 0) TL(4, qt);
+            tc_fence_after();
+            const uint32_t sadr = lane_base + a_col(qt);
+            uint32_t s[128];
+            tmem_ld32_at<0>(sadr, s);
+            tmem_ld32_at<32>(sadr + 32, s);
+            tmem_ld32_at<64>(sadr + 64, s);
+            tmem_ld32_at<96>(sadr + 96, s);
+            tmem_ld_wait();
+            if (row == 0) TL(14, qt);
+            if (limit < 127) { // the query's own block: keys after the query are invisible
 #pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (c > limit) s[c] = kNegInfBits;
-                }
-                float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F;
-#pragma unroll
-                for (int c = 0; c < 128; c += 4) {
-                    m0 = max3f(m0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-                    m1 = max3f(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-                }
-                const float m = fmaxf(m0, m1);
-                const uint64_t sl2x2 = f2_pack(sl2, sl2);
-                const uint64_t nmx2 = f2_pack(-m * sl2, -m * sl2);
-                uint64_t l2 = 0;
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int c = c4 * 32 + 2 * q;
-                        const uint64_t xx = f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2x2,
-                                                   nmx2);
-                        const float e0 = ex2_approx(f2_lo(xx)), e1 = ex2_approx(f2_hi(xx));
-                        l2 = f2_add(l2, f2_pack(e0, e1));
-                        pk[q] = pack_bf16x2(e0, e1);
-                    }
-                    tmem_st16(sadr + c4 * 16, pk);
-                }
-                sh.ml[qt & 3][row] = make_float2(m, f2_lo(l2) + f2_hi(l2));
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&sh.p_full[qa]);
-                    mbar_arrive(&sh.ml_full[qt & 3]);
-                }
-                if (row == 0) TL(5, qt);
+                for (int c = 0; c < 128; ++c)
+                    if (c > limit) s[c] = kNegInfBits;
             }
+            float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F;
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+                m0 = max3f(m0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                m1 = max3f(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+            }
+            const float m = fmaxf(m0, m1);
+            const uint64_t sl2x2 = f2_pack(sl2, sl2);
+            const uint64_t nmx2 = f2_pack(-m * sl2, -m * sl2);
+            uint64_t l2 = 0;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int c = c4 * 32 + 2 * q;
+                    const uint64_t xx = f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2x2,
+                                               nmx2);
+                    const float e0 = ex2_approx(f2_lo(xx)), e1 = ex2_approx(f2_hi(xx));
+                    l2 = f2_add(l2, f2_pack(e0, e1));
+                    pk[q] = pack_bf16x2(e0, e1);
+                }
+                tmem_st16(sadr + c4 * 16, pk);
+            }
+            sh.ml[qt & 3][row] = make_float2(m, f2_lo(l2) + f2_hi(l2));
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sh.p_full[qa]);
+                mbar_arrive(&sh.ml_full[qt & 3]);
+            }
+            if (row == 0) TL(5, qt);
         }
     } else {
         reg_set<REG_EPILOGUE, REG_LAUNCH>();
@@ -355,68 +406,65 @@ __global__ void __launch_bounds__(512, 1)
         const int pl = row / G, hh = row % G;
         const float scale = rsqrtf((float)DH);
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        int qt = 0;
-        bool ok = true;
-        for (int j = j_begin; j < j_end && ok; j += P) {
-            const msa_work_item item = a.items[j];
-            const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
-            const int ntiles = (item.len + PPT - 1) / PPT;
-            for (int t = 0; t < ntiles; ++t, ++qt) {
-                if (row == 0) TL(15, qt);
-                const int idx = t * PPT + pl;
-                const bool valid = idx < item.len;
-                const int32_t e = valid ? ent[idx] : 0;
-                const int p = e / a.k;
-                const int slot = e - p * a.k;
-                if (!wait_or_abort(&sh.o_full[qt & 1], (qt >> 1) & 1, abort_flag, a.err, 27, kWaitLimit) ||
-                    !wait_or_abort(&sh.ml_full[qt & 3], (qt >> 2) & 1, abort_flag, a.err, 29, kWaitLimit)) {
-                    ok = false;
-                    break;
-                }
-                if (row == 0) TL(6, qt);
-                tc_fence_after();
-                const float2 ml = sh.ml[qt & 3][row];
-                const float inv_l = 1.f / ml.y;
-                const int h = item.r * G + hh;
-                const int64_t prow = (int64_t)(p - a.row0);
-                bool store = valid;
-                if (valid && (prow < 0 || prow >= a.rows_pass || slot < 0 || slot >= a.k)) {
-                    report_error(a.err, MSA_ERR_DEVICE_CHECK, 300); // entry outside this pass: skip it
-                    store = false;
-                }
-                // partial layout [row][slot][d_h/8][H_q][8]: the G heads of a position are adjacent
-                // 16-byte units, so each warp-wide store writes contiguous runs
-                uint4* d4 = reinterpret_cast<uint4*>(a.o_part + (prow * a.k + slot) * (int64_t)a.H_q * DH) + h;
-                const uint64_t il2 = f2_pack(inv_l, inv_l);
-#pragma unroll
-                for (int c = 0; c < DH / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + o_col(qt) + c * 32, o);
-                    tmem_ld_wait();
-                    if (c == DH / 32 - 1) { // O fully read: PV of the next tile may overwrite it
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sh.o_free[qt & 1]);
-                        if (row == 0) TL(13, qt);
-                    }
-                    if (store) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int z = 0; z < 4; ++z) {
-                                const uint64_t y = f2_mul(
-                                    f2_pack(__uint_as_float(o[8 * q + 2 * z]), __uint_as_float(o[8 * q + 2 * z + 1])),
-                                    il2);
-                                w[z] = pack_bf16x2(f2_lo(y), f2_hi(y));
-                            }
-                            d4[(c * 4 + q) * a.H_q] = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                    }
-                }
-                if (store) a.lse_part[(prow * a.k + slot) * a.H_q + h] = ml.x * scale + logf(ml.y);
-                if (row == 0) TL(7, qt);
+        for (int qt = 0;; ++qt) {
+            if (row == 0) TL(15, qt);
+            const int rs = qt % kRing;
+            if (!wait_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 37, kWaitLimit)) break;
+            const TileRec rec = sh.rec[rs];
+            if (rec.npos < 0) break;
+            const bool valid = pl < rec.npos;
+            const int32_t e = valid ? sh.rec_e[rs][pl] : 0;
+            const int p = e / a.k;
+            const int slot = e - p * a.k;
+            if (!wait_or_abort(&sh.o_full[qt & 1], (qt >> 1) & 1, abort_flag, a.err, 27, kWaitLimit) ||
+                !wait_or_abort(&sh.ml_full[qt & 3], (qt >> 2) & 1, abort_flag, a.err, 29, kWaitLimit))
+                break;
+            if (row == 0) TL(6, qt);
+            tc_fence_after();
+            const float2 ml = sh.ml[qt & 3][row];
+            const float inv_l = 1.f / ml.y;
+            const int h = rec.r * G + hh;
+            const int64_t prow = (int64_t)(p - a.row0);
+            bool store = valid;
+            if (valid && (prow < 0 || prow >= a.rows_pass || slot < 0 || slot >= a.k)) {
+                report_error(a.err, MSA_ERR_DEVICE_CHECK, 300); // entry outside this pass: skip it
+                store = false;
             }
+            // partial layout [row][slot][d_h/8][H_q][8]: the G heads of a position are adjacent
+            // 16-byte units, so each warp-wide store writes contiguous runs
+            uint4* d4 = reinterpret_cast<uint4*>(a.o_part + (prow * a.k + slot) * (int64_t)a.H_q * DH) + h;
+            const uint64_t il2 = f2_pack(inv_l, inv_l);
+#pragma unroll
+            for (int c = 0; c < DH / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + o_col(qt) + c * 32, o);
+                tmem_ld_wait();
+                if (c == DH / 32 - 1) { // O fully read: PV of the next tile may overwrite it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&sh.o_free[qt & 1]);
+                        mbar_arrive(&sh.tile_free[rs]); // S, softmax and PV of qt are done with the record
+                    }
+                    if (row == 0) TL(13, qt);
+                }
+                if (store) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int z = 0; z < 4; ++z) {
+                            const uint64_t y = f2_mul(
+                                f2_pack(__uint_as_float(o[8 * q + 2 * z]), __uint_as_float(o[8 * q + 2 * z + 1])),
+                                il2);
+                            w[z] = pack_bf16x2(f2_lo(y), f2_hi(y));
+                        }
+                        d4[(c * 4 + q) * a.H_q] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+            if (store) a.lse_part[(prow * a.k + slot) * a.H_q + h] = ml.x * scale + logf(ml.y);
+            if (row == 0) TL(7, qt);
         }
     }
 
