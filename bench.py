@@ -42,6 +42,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["msa", "reference"], default="msa")
     ap.add_argument("--workload", default=synth.P128K.name, choices=sorted(synth.PREFILL_CONFIGS))
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-workload", default=synth.DECODE64.name, choices=sorted(synth.DECODE_CONFIGS))
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-oracle sample time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -56,6 +57,33 @@ def load_peaks():
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
                 "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu capture of a smaller case of
+# the same kernel, per query row of the launch; partial outputs grow in proportion to the rows, so a
+# full launch is the per-row figure times its rows. A figure only applies to the sources it was
+# measured on: after any change to them the bench reports traffic as null.
+PROFILED_TRAFFIC = {
+    "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "5d02559ac652877b",
+             "bytes_per_row": 320707.6, "capture": "profiles/sparse_attn_prefill_N32768.md (8192-row pass)"},
+    "combine": {"files": ("combine.cu", "common.cuh", "sm100.cuh"), "sha256_16": "bc1d0ab87cb62688",
+                "bytes_per_row": 282412.2, "capture": "profiles/combine_prefill_N32768.md (8192-row pass)"},
+}
+
+
+def profiled_traffic(name, rows_per_launch):
+    t = PROFILED_TRAFFIC.get(name)
+    if t is None:
+        return None
+    import hashlib
+
+    m = hashlib.sha256()
+    for f in t["files"]:
+        with open(os.path.join(ROOT, "block_sparse_long_idx_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    if m.hexdigest()[:16] != t["sha256_16"]:
+        return None
+    return t["bytes_per_row"] * rows_per_launch
 
 
 # ------------------------------------------------------------------------------------ CPU oracle
@@ -121,12 +149,41 @@ def workload_config(cfg, dcfg):
 
 
 class ClockSampler:
+    """Samples SM clock, power and clock-event reasons during the timed region: NVML every 10 ms
+    (read-only queries), or `nvidia-smi -lms 50` when the NVML bindings are missing."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
+
     def __init__(self, uuid: str):
         self.uuid = uuid
+        self.samples = []  # (sm_mhz, max_mhz, reason bits)
+        self.stop = threading.Event()
         self.proc = None
-        self.lines = []
+        self.t = None
 
     def __enter__(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+
+            def poll():
+                while not self.stop.is_set():
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((float(sm), float(mx), int(rs)))
+                    except pynvml.NVMLError:
+                        pass
+                    self.stop.wait(0.01)
+
+            self.t = threading.Thread(target=poll, daemon=True)
+            self.t.start()
+            return self
+        except Exception:  # no NVML bindings: fall back to nvidia-smi
+            pass
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -134,42 +191,43 @@ class ClockSampler:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={q}",
                                           "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t = threading.Thread(target=self._read_smi, daemon=True)
             self.t.start()
         except OSError:
             self.proc = None
         return self
 
-    def _read(self):
+    def _read_smi(self):
+        bits = [0x8, 0x40, 0x20, 0x4]
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            f = [x.strip() for x in line.strip().split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rs = sum(b for b, v in zip(bits, f[5:9]) if v.lower() == "active")
+                self.samples.append((float(f[1]), float(f[2]), rs))
+            except ValueError:
+                continue
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.t:
+            self.t.join(timeout=5)
         return False
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({nm for _, _, rs in self.samples for b, nm in self.REASONS.items() if rs & b})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_min_mhz": min(sm) if sm else None,
+                "sm_max_mhz": self.samples[-1][1] if self.samples else None, "reasons": reasons,
+                "samples": len(sm), "source": "nvml" if self.proc is None else "nvidia-smi"}
 
 
 def gpu_arm(args, rank, world):
@@ -184,7 +242,8 @@ def gpu_arm(args, rank, world):
     peaks = load_peaks()
     cfg = synth.PREFILL_CONFIGS[args.workload]
     cfg = cfg.with_(seed=replicas.replica_seed(cfg.seed, rank))  # independent sequence per rank
-    dcfg = None if args.no_decode else synth.DECODE64.with_(seed=replicas.replica_seed(synth.DECODE64.seed, rank))
+    dbase = synth.DECODE_CONFIGS[args.decode_workload]
+    dcfg = None if args.no_decode else dbase.with_(seed=replicas.replica_seed(dbase.seed, rank))
 
     host = synth.prefill_inputs(cfg)
     cpu_base = None
@@ -320,12 +379,20 @@ def gpu_arm(args, rank, world):
                 ach = work / (per_step / 1000.0) / 1e9
                 ent.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "peak": peaks["hbm_gbs"],
                             "frac": ach / peaks["hbm_gbs"], "algorithmic": work})
+        if name in ("attn", "combine"):
+            rows = N / max(1.0, ent["launches_per_step"])
+            tr = profiled_traffic(name, rows)
+            ent["traffic"] = tr
+            if tr is not None:
+                ent["traffic_source"] = PROFILED_TRAFFIC[name]["capture"] + ", scaled by rows per launch"
         kstats[name] = ent
     # dominant kernel of the prefill step
     dom = max((n for n in ("index_topk", "attn", "combine") if n in kstats), key=lambda n: kstats[n]["ms_per_step"])
     d = kstats[dom]
     roof = {"kernel": dom, "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
-            "frac": d["frac"], "traffic": None, "peak_source": peaks["source"] + " (burst)"}
+            "frac": d["frac"], "traffic": d.get("traffic"), "peak_source": peaks["source"] + " (burst)"}
+    if d.get("traffic") is not None:
+        roof["traffic_source"] = d["traffic_source"]
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": (pf_total + dec_total) / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

@@ -165,8 +165,12 @@ P128K = PrefillConfig("planted_prefill_N131072", N=131072, H_q=64, H_kv=4, d_h=1
 P1M = PrefillConfig("prefill_N1048576", N=1048576, H_q=64, H_kv=4, d_h=128, d_idx=64, B_k=128, k=16, seed=3)
 DECODE64 = DecodeConfig("decode_B64_L16K-128K", B=64, L_max=131072, len_lo=16384, len_hi=131072, H_q=64, H_kv=4,
                         d_h=128, d_idx=64, B_k=128, k=16, seed=4)
+# the same decode step over shorter caches (2 GB of K/V): small enough for detailed profiler captures
+DECODE64_SHORT = DecodeConfig("decode_B64_L2K-16K", B=64, L_max=16384, len_lo=2048, len_hi=16384, H_q=64, H_kv=4,
+                              d_h=128, d_idx=64, B_k=128, k=16, seed=5)
 
 PREFILL_CONFIGS = {c.name: c for c in (TINY, P32K, P128K, P1M)}
+DECODE_CONFIGS = {c.name: c for c in (DECODE64, DECODE64_SHORT)}
 
 
 # --------------------------------------------------------------------------
