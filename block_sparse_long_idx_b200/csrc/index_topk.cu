@@ -149,13 +149,13 @@ __global__ void __launch_bounds__(384, 1)
                 int r, u, steps;
                 bool tbv;
                 item_of(j, n_pairs, a.H_kv, n_qt, r, u, tbv, steps);
-                if (!wait_or_abort(&sh.q_full, item_cnt & 1, abort_flag, a.err, 3, kWaitLimit)) break;
+                if (!poll_or_abort(&sh.q_full, item_cnt & 1, abort_flag, a.err, 3, kWaitLimit)) break;
                 tc_fence_after();
                 for (int b = 0; b < steps; ++b, ++gstep, ++acc_cnt) {
                     const int s = gstep % C::NST;
                     const int buf = acc_cnt & 1;
-                    if (!wait_or_abort(&sh.kv_full[s], (gstep / C::NST) & 1, abort_flag, a.err, 4, kWaitLimit) ||
-                        !wait_or_abort(&sh.acc_empty[buf], ((acc_cnt >> 1) & 1) ^ 1, abort_flag, a.err, 5, kWaitLimit)) {
+                    if (!poll_or_abort(&sh.kv_full[s], (gstep / C::NST) & 1, abort_flag, a.err, 4, kWaitLimit) ||
+                        !poll_or_abort(&sh.acc_empty[buf], ((acc_cnt >> 1) & 1) ^ 1, abort_flag, a.err, 5, kWaitLimit)) {
                         ok = false;
                         break;
                     }
@@ -213,17 +213,13 @@ __global__ void __launch_bounds__(384, 1)
                         tmem_ld_wait();
 #pragma unroll
                         for (int c = 0; c < 32; c += 4) {
-                            m0 = fmaxf(m0, __uint_as_float(x[c]));
-                            m1 = fmaxf(m1, __uint_as_float(x[c + 1]));
-                            m2 = fmaxf(m2, __uint_as_float(x[c + 2]));
-                            m3 = fmaxf(m3, __uint_as_float(x[c + 3]));
-                            m0 = fmaxf(m0, __uint_as_float(y[c]));
-                            m1 = fmaxf(m1, __uint_as_float(y[c + 1]));
-                            m2 = fmaxf(m2, __uint_as_float(y[c + 2]));
-                            m3 = fmaxf(m3, __uint_as_float(y[c + 3]));
+                            m0 = max3f(m0, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+                            m1 = max3f(m1, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+                            m2 = max3f(m2, __uint_as_float(y[c]), __uint_as_float(y[c + 1]));
+                            m3 = max3f(m3, __uint_as_float(y[c + 2]), __uint_as_float(y[c + 3]));
                         }
                     }
-                    list.offer(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), b);
+                    list.offer_ascending(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), b); // blocks arrive in ascending order
                 }
                 tc_fence_before();
                 __syncwarp();

@@ -62,6 +62,26 @@ struct TopkList {
     {
         if (admits(val, blk)) insert(val, blk);
     }
+
+    // offer() for a block whose index exceeds that of every listed block (a row's blocks offered in
+    // ascending order): an equal score never beats a listed one, so the order test is a strict
+    // greater-than, and the insertion becomes one independent select per slot (slot j takes its
+    // left neighbour if val beats that, else val if val beats slot j, else keeps its entry) instead
+    // of a serial shift. Sentinels (+inf) are never displaced.
+    __device__ __forceinline__ void offer_ascending(float val, int blk)
+    {
+        if (!(val > v[L - 1])) return;
+        bool c[L];
+#pragma unroll
+        for (int j = 0; j < L; ++j) c[j] = val > v[j];
+#pragma unroll
+        for (int j = L - 1; j >= 1; --j) {
+            v[j] = c[j - 1] ? v[j - 1] : (c[j] ? val : v[j]);
+            b[j] = c[j - 1] ? b[j - 1] : (c[j] ? blk : b[j]);
+        }
+        v[0] = c[0] ? val : v[0];
+        b[0] = c[0] ? blk : b[0];
+    }
 };
 
 // Final selection of one (row, group): the admitted blocks plus the local block, ascending,
