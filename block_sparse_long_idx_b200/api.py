@@ -54,6 +54,8 @@ SIGNATURES = [
     ("msa_sparse_decode_workspace_size", _sz, [_int, _i64, _int, _int, _int, _int, _int, _int]),
     ("msa_sparse_decode", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _int, _int, _int, _vp,
                                  _vp, _vp, _vp, _sz, _vp]),
+    ("msa_selftest_workspace_size", _sz, []),
+    ("msa_selftest_wait_timeout", _int, [_vp, _sz, _i64, _vp]),
     ("msa_trace_set", None, [_vp]),
     ("msa_last_error_string", ctypes.c_char_p, []),
     ("msa_launch_count", ctypes.c_uint64, []),
@@ -157,6 +159,16 @@ def status_string(status: int) -> str:
 def msa_get_device_error(workspace: torch.Tensor, stream=None) -> int:
     """Device error word of a workspace used by a previous call (synchronises the stream)."""
     return lib.msa_get_device_error(workspace.data_ptr(), _stream(stream))
+
+
+def msa_selftest_wait_timeout(limit_cycles: int = 1_000_000, workspace=None, device=None, stream=None) -> int:
+    """Runs the bounded-wait failure path on the device (a wait that can never complete) and
+    returns the device status it left: MSA_ERR_TIMEOUT when the path works."""
+    dev = workspace.device if workspace is not None else (device or torch.device("cuda"))
+    ws = _workspace(lib.msa_selftest_workspace_size(), dev, workspace)
+    _check("msa_selftest_wait_timeout", lib.msa_selftest_wait_timeout(ws.data_ptr(), ws.numel(), int(limit_cycles),
+                                                                       _stream(stream)))
+    return msa_get_device_error(ws, stream)
 
 
 def msa_index_topk(q_idx, k_idx, B_k: int = 128, k: int = 16, block_idx=None, workspace=None, stream=None):

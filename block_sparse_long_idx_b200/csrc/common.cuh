@@ -83,6 +83,9 @@ struct AttnArgs {
     float* lse_part;            // [rows][k][H_q]
     int* err;
 };
+// One thread waits on a barrier phase that never completes; the wait expires after limit_cycles.
+cudaError_t launch_selftest_wait(int* err, long long limit_cycles, cudaStream_t s);
+
 cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                                const CUtensorMap& vmap, cudaStream_t s);
 

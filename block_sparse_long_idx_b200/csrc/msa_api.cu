@@ -142,6 +142,21 @@ msa_status msa_get_device_error(const void* workspace, msa_stream_t stream)
     return (msa_status)h[0];
 }
 
+// ------------------------------------------------------------------------------------ self-test
+size_t msa_selftest_workspace_size(void) { return kErrBytes; }
+
+msa_status msa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,
+                                     msa_stream_t stream)
+{
+    if (!workspace || !aligned(workspace, 256) || limit_cycles < 1 || limit_cycles > 2000000000LL)
+        return MSA_ERR_INVALID_ARG;
+    if (workspace_bytes < kErrBytes) return MSA_ERR_WORKSPACE;
+    if (injected("msa_selftest_wait_timeout")) return MSA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    return cuda_status(launch_selftest_wait((int*)workspace, (long long)limit_cycles, s), "self-test launch");
+}
+
 // ------------------------------------------------------------------------------------ index_topk
 size_t msa_index_topk_workspace_size(int64_t, int, int, int, int) { return kErrBytes; }
 

@@ -74,6 +74,21 @@ MSA_API const char* msa_last_error_string(void);
  */
 MSA_API msa_status msa_get_device_error(const void* workspace, msa_stream_t stream);
 
+/*
+ * Failure-path self-test (a diagnostic; the pages have no counterpart). Launches one thread that
+ * waits, through the same bounded-wait routine every kernel of this library uses, on a barrier
+ * phase that nothing completes. After `limit_cycles` SM clock cycles the wait gives up, records
+ * MSA_ERR_TIMEOUT in the device error word at the start of `workspace` and the kernel returns:
+ * msa_get_device_error() then reports MSA_ERR_TIMEOUT and the CUDA context stays usable.
+ *   workspace       : >= msa_selftest_workspace_size() bytes, 256-byte aligned, caller-owned
+ *   limit_cycles    : 1 .. 2,000,000,000 (about one second of SM clock at the upper end)
+ * Returns MSA_ERR_INVALID_ARG / MSA_ERR_WORKSPACE before enqueueing anything, MSA_ERR_CUDA if the
+ * launch failed, else MSA_OK (the timeout itself is read with msa_get_device_error).
+ */
+MSA_API size_t msa_selftest_workspace_size(void);
+MSA_API msa_status msa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,
+                                             msa_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Index Branch: fused index score + block max-pool + exp-free Top-k      [EXPL Fig. 1, 05-1]
  *

@@ -106,3 +106,14 @@ def test_host_fault_injection():
     env = dict(os.environ, MSA_FAULT_INJECT="msa_index_topk")
     out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert "STATUS 4" in out.stdout, out.stdout + out.stderr
+
+
+def test_selftest_validation(msa):
+    """The failure-path self-test rejects bad arguments before launching anything."""
+    lib = msa.lib
+    assert lib.msa_selftest_workspace_size() >= 8
+    assert lib.msa_selftest_wait_timeout(None, 256, 1000, None) == INVALID
+    assert lib.msa_selftest_wait_timeout(WS + 8, 256, 1000, None) == INVALID  # not 256-byte aligned
+    assert lib.msa_selftest_wait_timeout(WS, 256, 0, None) == INVALID
+    assert lib.msa_selftest_wait_timeout(WS, 256, 2_000_000_001, None) == INVALID
+    assert lib.msa_selftest_wait_timeout(WS, 8, 1000, None) == WORKSPACE
