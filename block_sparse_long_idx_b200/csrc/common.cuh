@@ -112,6 +112,7 @@ struct DecodeArgs {
     int64_t L_max;
     int H_q, H_kv, d_h, d_idx, k;
     float* pooled;        // [B][H_kv][nb_max]
+    int64_t* blk_prefix;  // [B + 1] fully visible blocks of the sequences before beta
     int32_t* sel;         // [B][H_kv][k]
     int32_t* nsel;        // [B]
     uint16_t* o_part;     // [B][k][H_q][d_h]

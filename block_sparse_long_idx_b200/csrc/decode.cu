@@ -25,17 +25,57 @@ namespace msa {
 namespace {
 
 constexpr int kPoolWarps = 8;
-constexpr int kPoolSplits = 16;
+constexpr int kPoolCtasPerSm = 8;
 
 __device__ __forceinline__ int seq_local_block(int len) { return (len - 1) / kBk; }
 
 // ----------------------------------------------------------------------------------- 1. pooling
+// Work balance: sequences have very different lengths, so the fully visible blocks of all
+// sequences form one flattened list (prefix[beta] = blocks of the sequences before beta) and every
+// warp of a persistent grid streams an equal contiguous slice of it.
+__global__ void __launch_bounds__(1024) decode_prefix_kernel(DecodeArgs a)
+{
+    __shared__ int64_t warp_sum[32];
+    __shared__ int64_t carry;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        carry = 0;
+        a.blk_prefix[0] = 0;
+    }
+    __syncthreads();
+    for (int base = 0; base < a.B; base += 1024) {
+        const int beta = base + tid;
+        int64_t n = 0;
+        if (beta < a.B) {
+            const int len = a.lens[beta];
+            n = (len >= 1 && len <= a.L_max) ? seq_local_block(len) : 0;
+        }
+        int64_t x = n; // inclusive scan: warp, then across warps
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sum[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int64_t w = warp_sum[lane];
+            for (int o = 1; o < 32; o <<= 1) {
+                const int64_t y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sum[lane] = w;
+        }
+        __syncthreads();
+        const int64_t incl = carry + x + (warp > 0 ? warp_sum[warp - 1] : 0);
+        if (beta < a.B) a.blk_prefix[beta + 1] = incl;
+        __syncthreads();
+        if (tid == 1023) carry = incl;
+        __syncthreads();
+    }
+}
+
 __global__ void __launch_bounds__(kPoolWarps * 32) decode_pool_kernel(DecodeArgs a, int nb_max)
 {
-    const int beta = blockIdx.x;
-    const int len = a.lens[beta];
-    if (len < 1 || len > a.L_max) return; // reported by decode_topk
-    const int n_cand = seq_local_block(len); // fully visible non-local blocks
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int lanes_per_pos = (a.H_kv * a.d_idx) / 8;
     const int pos_per_step = 32 / lanes_per_pos;
@@ -43,33 +83,68 @@ __global__ void __launch_bounds__(kPoolWarps * 32) decode_pool_kernel(DecodeArgs
     const int sub = lane % lanes_per_pos;
     const int r = sub / lanes_per_group;
     const int pos_lane = lane / lanes_per_pos;
-    // this lane's 8 query elements
-    const uint4 qv = *reinterpret_cast<const uint4*>(a.q_idx + ((int64_t)beta * a.H_kv) * a.d_idx + sub * 8);
-    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-    float qf[8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        qf[2 * q] = __uint_as_float(qw[q] << 16);
-        qf[2 * q + 1] = __uint_as_float(qw[q] & 0xFFFF0000u);
-    }
     const int64_t row_elems = (int64_t)a.H_kv * a.d_idx;
-    const uint16_t* cache = a.k_idx_cache + (int64_t)beta * a.L_max * row_elems + sub * 8;
-    for (int b = blockIdx.y * kPoolWarps + warp; b < n_cand; b += kPoolSplits * kPoolWarps) {
-        float m = -CUDART_INF_F;
-        const uint16_t* blk = cache + (int64_t)b * kBk * row_elems;
-#pragma unroll 4
-        for (int j0 = 0; j0 < kBk; j0 += pos_per_step) {
-            const int j = j0 + pos_lane;
-            const uint4 kv = __ldg(reinterpret_cast<const uint4*>(blk + (int64_t)j * row_elems));
-            const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-            float s = 0.f;
+    const int64_t total = a.blk_prefix[a.B];
+    const int64_t n_warps = (int64_t)gridDim.x * kPoolWarps;
+    const int64_t wid = (int64_t)blockIdx.x * kPoolWarps + warp;
+    const int64_t g0 = total * wid / n_warps, g1 = total * (wid + 1) / n_warps;
+    if (g0 >= g1) return;
+    // the sequence holding block g0: the last beta with prefix[beta] <= g0
+    int lo = 0, hi = a.B - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.blk_prefix[mid] <= g0) lo = mid; else hi = mid - 1;
+    }
+    int beta = -1;
+    int64_t seq_begin = 0, seq_end = 0;
+    float qf[8];
+    const uint16_t* cache = nullptr;
+    for (int64_t g = g0; g < g1; ++g) {
+        if (g >= seq_end) { // enter the next sequence that owns blocks (empty ones are skipped)
+            beta = beta < 0 ? lo : beta + 1;
+            while (a.blk_prefix[beta + 1] <= g) ++beta;
+            seq_begin = a.blk_prefix[beta];
+            seq_end = a.blk_prefix[beta + 1];
+            const uint4 qv = *reinterpret_cast<const uint4*>(a.q_idx + ((int64_t)beta * a.H_kv) * a.d_idx + sub * 8);
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                s = fmaf(qf[2 * q], __uint_as_float(kw[q] << 16), s);
-                s = fmaf(qf[2 * q + 1], __uint_as_float(kw[q] & 0xFFFF0000u), s);
+                qf[2 * q] = __uint_as_float(qw[q] << 16);
+                qf[2 * q + 1] = __uint_as_float(qw[q] & 0xFFFF0000u);
             }
-            for (int o = lanes_per_group >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            m = fmaxf(m, s);
+            cache = a.k_idx_cache + (int64_t)beta * a.L_max * row_elems + sub * 8;
+        }
+        const int b = (int)(g - seq_begin);
+        float m = -CUDART_INF_F;
+        const uint16_t* blk = cache + (int64_t)b * kBk * row_elems;
+        // 8 cache rows in flight per warp: issue the loads, then reduce
+        for (int j0 = 0; j0 < kBk; j0 += 8 * pos_per_step) {
+            uint4 kv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + u * pos_per_step + pos_lane;
+                kv[u] = j < kBk ? __ldg(reinterpret_cast<const uint4*>(blk + (int64_t)j * row_elems))
+                                : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float s[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t kw[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+                float acc = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc = fmaf(qf[2 * q], __uint_as_float(kw[q] << 16), acc);
+                    acc = fmaf(qf[2 * q + 1], __uint_as_float(kw[q] & 0xFFFF0000u), acc);
+                }
+                s[u] = acc;
+            }
+            for (int o = lanes_per_group >> 1; o > 0; o >>= 1) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (j0 + u * pos_per_step < kBk) m = fmaxf(m, s[u]);
         }
         for (int o = lanes_per_pos; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane < lanes_per_pos && (sub % lanes_per_group) == 0)
@@ -330,13 +405,17 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s)
 {
     const int nb_max = (int)((a.L_max + kBk - 1) / kBk);
+    int dev = 0, n_sm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     trace_begin(s);
-    decode_pool_kernel<<<dim3(a.B, kPoolSplits), kPoolWarps * 32, 0, s>>>(a, nb_max);
+    decode_prefix_kernel<<<1, 1024, 0, s>>>(a);
+    decode_pool_kernel<<<n_sm * kPoolCtasPerSm, kPoolWarps * 32, 0, s>>>(a, nb_max);
     trace_end(s, MSA_KERNEL_DEC_POOL);
     trace_begin(s);
     decode_topk_kernel<<<dim3(a.B, a.H_kv), 32, 0, s>>>(a, nb_max);
     trace_end(s, MSA_KERNEL_DEC_TOPK);
-    note_launch(3);
+    note_launch(4);
     trace_begin(s);
     cudaError_t e;
     if (a.d_h == 128) {

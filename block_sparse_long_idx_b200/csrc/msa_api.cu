@@ -416,6 +416,7 @@ size_t msa_sparse_decode_workspace_size(int B, int64_t L_max, int H_q, int H_kv,
     sz += align_up((size_t)B * 4, 256);
     sz += align_up((size_t)B * k * H_q * d_h * 2, 256);
     sz += align_up((size_t)B * k * H_q * 4, 256);
+    sz += align_up((size_t)(B + 1) * 8, 256);
     return sz;
 }
 
@@ -470,6 +471,8 @@ msa_status msa_sparse_decode(const msa_bf16* q, const msa_bf16* q_idx, const msa
     a.o_part = (uint16_t*)(ws + off);
     off += align_up((size_t)B * k * H_q * d_h * 2, 256);
     a.lse_part = (float*)(ws + off);
+    off += align_up((size_t)B * k * H_q * 4, 256);
+    a.blk_prefix = (int64_t*)(ws + off);
     a.out = out;
     a.lse = lse;
     a.block_idx_out = block_idx_out;
