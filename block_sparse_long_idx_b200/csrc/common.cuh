@@ -77,6 +77,7 @@ struct AttnArgs {
     int w0, w1;                 // windows of this pass
     int64_t row0;               // first row of the pass (= w0 * window)
     int64_t rows_pass;          // rows the partial buffers hold
+    int* item_counter;          // work items claimed so far in this launch (zero at launch)
     long long* timeline;        // optional: CTA 0 records clock64 per tile event (nullptr = off)
     int timeline_tiles;         // capacity in tiles (16 event slots per tile)
     uint16_t* o_part;           // [rows][k][H_q][d_h]

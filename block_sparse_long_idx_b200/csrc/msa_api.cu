@@ -376,11 +376,14 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
         a.w1 = (int)w1;
         a.row0 = w0 * L->window;
         a.rows_pass = rows_pass;
+        a.item_counter = (int*)workspace + 4; // inside the error-word region, reset for every pass
         a.timeline = nullptr;
         a.timeline_tiles = 0;
         a.o_part = o_part;
         a.lse_part = lse_part;
         a.err = (int*)workspace;
+        if (msa_status st1 = cuda_status(cudaMemsetAsync(a.item_counter, 0, sizeof(int), s), "clearing the work counter"))
+            return st1;
         trace_begin(s);
         const cudaError_t ea = launch_sparse_attn(a, qmap, kmap, vmap, s);
         trace_end(s, MSA_KERNEL_ATTN);

@@ -17,10 +17,13 @@
 // Roles (512 threads, four warpgroups):
 //   WG0: warp 0 = K/V TMA producer, warp 1 = S issuer + TMEM owner, warp 2 = tile scheduler and Q
 //        gather (one TMA box per position, issued by the 32 lanes in parallel), warp 3 = PV issuer
-// The tile scheduler is the only role that reads the work list in global memory after the K/V
-// producer: it publishes every tile as a record (group, block, positions, their entries, item
-// boundaries) in a shared-memory ring that the MMA issuers, the softmax and the epilogue consume,
-// so none of them waits on a global load. The epilogue releases a record after its tile's PV.
+// Work items are claimed dynamically: the tile scheduler takes the next item of the launch's work
+// list from a global atomic counter (so CTAs that drew short items take more), one item ahead of
+// its own use, and hands it to the K/V producer through a 4-deep shared-memory item ring. It is the
+// only role that reads the work list and the entries in global memory: it publishes every tile as
+// a record (group, block, positions, their entries, item boundaries) in a shared-memory ring that
+// the MMA issuers, the softmax and the epilogue consume, so none of them waits on a global load.
+// The epilogue releases a record after its tile's PV.
 //   WG1, WG2: softmax of even / odd tiles
 //   WG3: epilogue of every tile (O / rowsum -> partial slot)
 // TMEM (512 columns): two 128-column S/P regions A[t % 2] at columns 0 and 128 (S, then P in
@@ -65,9 +68,11 @@ struct AttnShared {
     uint64_t o_full[2], o_free[2];
     uint64_t ml_full[4];
     uint64_t tile_full[kRing], tile_free[kRing];
+    uint64_t kvrec_full[4], kvrec_free[4];
     uint64_t done, done2;
     float2 ml[4][128]; // (row max of the raw scores, row sum of exp) per tile slot and row
     TileRec rec[kRing];
+    msa_work_item kvrec[4]; // items handed to the K/V producer (len = 0: no more work)
     int32_t rec_e[kRing][128]; // entry (i*k + slot) of each position of the tile
     uint32_t tmem_base;
     int abort_flag;
@@ -98,10 +103,10 @@ __global__ void __launch_bounds__(512, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wg = warp >> 2;
-    const int P = gridDim.x, cta = blockIdx.x;
+    const int cta = blockIdx.x;
     const int64_t Nk = a.N * a.k;
     volatile int* abort_flag = &sh.abort_flag;
-    const int j_begin = a.window_items[a.w0] + cta;
+    const int j_base = a.window_items[a.w0];
     const int j_end = a.window_items[a.w1];
     const bool tl_on = a.timeline != nullptr && cta == 0;
 #define TL(slot, tile)                                                                                    \
@@ -130,6 +135,10 @@ __global__ void __launch_bounds__(512, 1)
             mbar_init(&sh.tile_full[i], 1);
             mbar_init(&sh.tile_free[i], 4);
         }
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&sh.kvrec_full[i], 1);
+            mbar_init(&sh.kvrec_free[i], 1);
+        }
         mbar_init(&sh.done, 1);
         mbar_init(&sh.done2, 1);
         sh.abort_flag = 0;
@@ -150,8 +159,12 @@ __global__ void __launch_bounds__(512, 1)
             // -------------------------------------------------------- K/V producer
             if (lane == 0) {
                 int it = 0;
-                for (int j = j_begin; j < j_end; j += P, ++it) {
-                    const msa_work_item item = a.items[j];
+                for (;; ++it) {
+                    const int s4 = it & 3;
+                    if (!wait_or_abort(&sh.kvrec_full[s4], (it >> 2) & 1, abort_flag, a.err, 38, kWaitLimit)) break;
+                    const msa_work_item item = sh.kvrec[s4];
+                    mbar_arrive(&sh.kvrec_free[s4]);
+                    if (item.len <= 0) break;
                     const int s = it & 1;
                     if (!wait_or_abort(&sh.kv_empty[s], ((it >> 1) & 1) ^ 1, abort_flag, a.err, 20, kWaitLimit))
                         break;
@@ -168,18 +181,36 @@ __global__ void __launch_bounds__(512, 1)
             }
         } else if (warp == 2) {
             // -------------------------------------------------------- tile scheduler + Q gather
-            int qt = 0, it = 0;
-            bool ok = true;
-            for (int j = j_begin; j < j_end && ok; j += P, ++it) {
-                const msa_work_item item = a.items[j];
-                if (item.len <= 0) { // the inversion never emits empty items; stop rather than desynchronise
-                    if (lane == 0) {
+            // claim the next work item and hand it to the K/V producer (record slot n & 3)
+            auto claim_and_publish = [&](int n, msa_work_item& item) -> bool {
+                int j = 0;
+                int w_ok = 1;
+                if (lane == 0) {
+                    j = j_base + atomicAdd(a.item_counter, 1);
+                    item = j < j_end ? a.items[j] : msa_work_item{0, 0, 0, 0};
+                    if (j < j_end && item.len <= 0) // the inversion never emits empty items: stop here
                         report_error(a.err, MSA_ERR_DEVICE_CHECK, 301);
-                        *abort_flag = 1;
+                    if (n >= 4)
+                        w_ok = wait_or_abort(&sh.kvrec_free[n & 3], ((n >> 2) & 1) ^ 1, abort_flag, a.err, 39,
+                                             kWaitLimit);
+                    if (w_ok) {
+                        sh.kvrec[n & 3] = item;
+                        mbar_arrive(&sh.kvrec_full[n & 3]);
                     }
-                    ok = false;
-                    break;
                 }
+                item.r = __shfl_sync(0xffffffffu, item.r, 0);
+                item.b = __shfl_sync(0xffffffffu, item.b, 0);
+                item.start = __shfl_sync(0xffffffffu, item.start, 0);
+                item.len = __shfl_sync(0xffffffffu, item.len, 0);
+                return __shfl_sync(0xffffffffu, w_ok, 0) != 0;
+            };
+            int qt = 0, it = 0;
+            msa_work_item item{0, 0, 0, 0};
+            bool ok = claim_and_publish(0, item);
+            while (ok && item.len > 0) {
+                msa_work_item next{0, 0, 0, 0};
+                ok = claim_and_publish(it + 1, next); // one item of look-ahead for the K/V producer
+                if (!ok) break;
                 const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
                 const int ntiles = (item.len + PPT - 1) / PPT;
                 for (int t = 0; t < ntiles; ++t, ++qt) {
@@ -235,6 +266,8 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     if (lane == 0) TL(1, qt);
                 }
+                item = next;
+                ++it;
             }
             const int n_tiles = qt;
             // two end records, so that each softmax warpgroup (even / odd tiles) meets one
