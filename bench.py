@@ -43,7 +43,7 @@ def parse_args():
     ap.add_argument("--workload", default=synth.P128K.name, choices=sorted(synth.PREFILL_CONFIGS))
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-workload", default=synth.DECODE64.name, choices=sorted(synth.DECODE_CONFIGS))
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-oracle sample time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows-per-pass", type=int, default=0, help="cap the prefill partial buffer (0 = whole N)")
@@ -64,9 +64,9 @@ def load_peaks():
 # full launch is the per-row figure times its rows. A figure only applies to the sources it was
 # measured on: after any change to them the bench reports traffic as null.
 PROFILED_TRAFFIC = {
-    "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "d7c8a9385d194bb3",
-             "bytes_per_row": 320707.6, "capture": "profiles/sparse_attn_prefill_N32768.md (8192-row pass)"},
-    "combine": {"files": ("combine.cu", "common.cuh", "sm100.cuh"), "sha256_16": "3d20cd4164dac1ee",
+    "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "b1c4a120f8dc8710",
+             "bytes_per_row": 307955.2, "capture": "profiles/sparse_attn_prefill_N32768.md (8192-row pass)"},
+    "combine": {"files": ("combine.cu", "common.cuh", "sm100.cuh"), "sha256_16": "930906627b9c1775",
                 "bytes_per_row": 282412.2, "capture": "profiles/combine_prefill_N32768.md (8192-row pass)"},
 }
 
@@ -130,7 +130,9 @@ def reference_arm(args, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(cfg, None),
+            "data": "synthetic",
+            "config": dict(workload_config(cfg, None if args.no_decode else synth.DECODE_CONFIGS[args.decode_workload]),
+                           parallelism=f"replicas x{args.gpus} (independent sequences)"),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": o.max_threads(), "kind": "oracle",
                              "sample": f"per step {rows_done[0]} sampled query rows of {cfg.name} "
                                        "(selection + attention, all heads)"},
@@ -278,12 +280,16 @@ def gpu_arm(args, rank, world):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def prefill():
-        msa.msa_index_topk(t["q_idx"], t["k_idx"], cfg.B_k, k, block_idx=block_idx, workspace=ws_idx)
+    def prefill(inp=None, dst=None):
+        inp = t if inp is None else inp
+        dst = out if dst is None else dst
+        cur = torch.cuda.current_stream()
+        msa.msa_index_topk(inp["q_idx"], inp["k_idx"], cfg.B_k, k, block_idx=block_idx, workspace=ws_idx, stream=cur)
         msa.api._check("msa_build_kv2q", msa.api.lib.msa_build_kv2q(
             block_idx.data_ptr(), msa.api.ctypes.byref(L), kv.buf.data_ptr(), ws_kv.data_ptr(), ws_kv.numel(),
-            stream.cuda_stream))
-        msa.msa_sparse_prefill(t["q"], t["k"], t["v"], block_idx, kv, out=out, lse=lse, workspace=ws_pf)
+            cur.cuda_stream))
+        msa.msa_sparse_prefill(inp["q"], inp["k"], inp["v"], block_idx, kv, out=dst, lse=lse, workspace=ws_pf,
+                               stream=cur)
 
     def decode():
         msa.msa_sparse_decode(dt["q"], dt["q_idx"], dt["k_cache"], dt["v_cache"], dt["k_idx_cache"], dt["lens"],
@@ -328,31 +334,58 @@ def gpu_arm(args, rank, world):
 
     pf_total, dec_total = replicas.max_over_ranks([sum(pf_ms), sum(dec_ms)], device=dev)
 
-    # end-to-end through the public API with host buffers (pinned), copies inside the timed region
+    # end-to-end through the public API with host buffers (pinned), copies inside the timed region:
+    # every step copies its inputs in and its output back; device inputs and outputs are double
+    # buffered so step s+1's inputs stream in and step s-1's output streams out while step s computes
     e2e = None
     if args.e2e_steps > 0:
         pin = {n: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory()
                for n, a in host.items()}
-        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        out_h = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
         h2d = sum(p.numel() * p.element_size() for p in pin.values())
-        d2h = out_h.numel() * out_h.element_size()
+        d2h = out_h[0].numel() * out_h[0].element_size()
+        dev_in = [t, {n: torch.empty_like(x) for n, x in t.items()}]
+        dev_out = [out, torch.empty_like(out)]
+        s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        in_ready = [torch.cuda.Event() for _ in range(args.e2e_steps)]
+        comp_done = [torch.cuda.Event() for _ in range(args.e2e_steps)]
+        out_done = [torch.cuda.Event() for _ in range(args.e2e_steps)]
+        flush.zero_()
+        torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        tot = 0.0
-        for s in range(args.e2e_steps):
-            flush.zero_()
-            e0.record()
-            for n in t:
-                t[n].copy_(pin[n], non_blocking=True)
-            prefill()
-            out_h.copy_(out, non_blocking=True)
-            e1.record()
-            torch.cuda.synchronize()
-            tot += e0.elapsed_time(e1)
-        (te,) = replicas.max_over_ranks([tot], device=dev)
+        e0.record(s_in)
+        s_comp.wait_event(e0)
+        s_out.wait_event(e0)
+        for st in range(args.e2e_steps):
+            bsel = st & 1
+            with torch.cuda.stream(s_in):
+                if st >= 2:
+                    s_in.wait_event(comp_done[st - 2])  # step st-2 has finished reading these inputs
+                for n in t:
+                    dev_in[bsel][n].copy_(pin[n], non_blocking=True)
+                in_ready[st].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(in_ready[st])
+                if st >= 2:
+                    s_comp.wait_event(out_done[st - 2])  # step st-2's output has been copied out
+                prefill(dev_in[bsel], dev_out[bsel])
+                comp_done[st].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[st])
+                out_h[bsel].copy_(dev_out[bsel], non_blocking=True)
+                out_done[st].record(s_out)
+        s_in.wait_stream(s_out)
+        s_in.wait_stream(s_comp)
+        e1.record(s_in)
+        torch.cuda.synchronize()
+        (te,) = replicas.max_over_ranks([e0.elapsed_time(e1)], device=dev)
         e2e = {"value": replicas.aggregate_rate(N * args.e2e_steps, world, te / 1000.0), "unit": UNIT,
                "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
-               "note": "prefill through the public API: pinned host inputs copied in, out copied back"}
+               "steps": args.e2e_steps,
+               "note": "prefill through the public API on host buffers: every step copies its inputs in from "
+                       "pinned memory and its output back; inputs/outputs double-buffered on the device so the "
+                       "copies of neighbouring steps overlap the current step's kernels"}
 
     if rank != 0:
         return

@@ -61,7 +61,6 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     with ThreadPoolExecutor(min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
     if force or _stale(LIB, objs):
-        cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", LIB + ".tmp"] + objs + ["-lcuda"]
         cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-Xcompiler", "-fPIC", "-o",
                LIB + ".tmp"] + objs
         if verbose:

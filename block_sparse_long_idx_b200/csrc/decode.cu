@@ -405,12 +405,17 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s)
 {
     const int nb_max = (int)((a.L_max + kBk - 1) / kBk);
-    int dev = 0, n_sm = 148;
+    int dev = 0, n_sm = 148, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    // one wave of resident CTAs: every warp gets an equal slice, so a second wave would only add a tail
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_pool_kernel, kPoolWarps * 32, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    if (per_sm > kPoolCtasPerSm) per_sm = kPoolCtasPerSm;
     trace_begin(s);
     decode_prefix_kernel<<<1, 1024, 0, s>>>(a);
-    decode_pool_kernel<<<n_sm * kPoolCtasPerSm, kPoolWarps * 32, 0, s>>>(a, nb_max);
+    decode_pool_kernel<<<n_sm * per_sm, kPoolWarps * 32, 0, s>>>(a, nb_max);
     trace_end(s, MSA_KERNEL_DEC_POOL);
     trace_begin(s);
     decode_topk_kernel<<<dim3(a.B, a.H_kv), 32, 0, s>>>(a, nb_max);
