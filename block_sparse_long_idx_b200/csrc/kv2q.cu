@@ -174,33 +174,42 @@ __global__ void kv2q_relative_kernel(Kv2qArgs a, const int32_t* group_starts)
 // ------------------------------------------------------------------------------------ 3. scatter
 __global__ void kv2q_scatter_kernel(Kv2qArgs a)
 {
-    extern __shared__ int32_t cur[];
+    extern __shared__ int32_t next_pos[]; // [nb] next write position of each block's list in this window
     const int w = blockIdx.x, r = blockIdx.y;
     const int lane = threadIdx.x;
-    for (int b = lane; b < a.nb; b += 32) cur[b] = 0;
+    const int32_t* bases = a.bases + (int64_t)r * a.nb * a.n_windows;
+    for (int b = lane; b < a.nb; b += 32) next_pos[b] = bases[(int64_t)b * a.n_windows + w];
     __syncwarp();
     const int64_t row_lo = (int64_t)w * a.window;
     const int64_t row_hi = min(a.N, row_lo + a.window);
     const int32_t* sel = a.block_idx + (int64_t)r * a.N * a.k;
     int32_t* ent = a.entries + (int64_t)r * a.N * a.k;
-    const int32_t* bases = a.bases + (int64_t)r * a.nb * a.n_windows;
     const int rows_per_step = 32 / a.k;
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int64_t i0 = row_lo; i0 < row_hi; i0 += rows_per_step) {
-        const int64_t i = i0 + lane / a.k;
-        const int slot = lane % a.k;
-        const bool in = lane < rows_per_step * a.k && i < row_hi;
-        int32_t b = in ? sel[i * a.k + slot] : -1;
-        if (b >= a.nb || (b >= 0 && (int64_t)b * kBk > i)) b = -1; // reported by the count pass
-        const unsigned peers = __match_any_sync(0xffffffffu, b);
-        if (b >= 0) {
-            const int rank = __popc(peers & lt_mask);
-            const int32_t pos = bases[(int64_t)b * a.n_windows + w] + cur[b] + rank;
-            ent[pos] = (int32_t)(i * a.k + slot);
+    const int slot = lane % a.k;
+    const bool lane_used = lane < rows_per_step * a.k;
+    constexpr int kAhead = 8; // selection loads in flight per lane
+    for (int64_t i00 = row_lo; i00 < row_hi; i00 += (int64_t)rows_per_step * kAhead) {
+        int32_t bs[kAhead];
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            const int64_t i = i00 + (int64_t)u * rows_per_step + lane / a.k;
+            bs[u] = lane_used && i < row_hi ? sel[i * a.k + slot] : -1;
         }
-        __syncwarp();
-        if (b >= 0 && (peers & lt_mask) == 0) cur[b] += __popc(peers);
-        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            const int64_t i = i00 + (int64_t)u * rows_per_step + lane / a.k;
+            int32_t b = bs[u];
+            if (b >= a.nb || (b >= 0 && (int64_t)b * kBk > i)) b = -1; // reported by the count pass
+            const unsigned peers = __match_any_sync(0xffffffffu, b);
+            if (b >= 0) {
+                const unsigned before = peers & lt_mask;
+                ent[next_pos[b] + __popc(before)] = (int32_t)(i * a.k + slot);
+                __syncwarp(peers);
+                if (before == 0) next_pos[b] += __popc(peers);
+            }
+            __syncwarp();
+        }
     }
 }
 
