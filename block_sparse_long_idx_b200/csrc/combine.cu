@@ -28,7 +28,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
     uint4* obuf = reinterpret_cast<uint4*>(csm + align_up_dev(a.k * a.H_q * 4)); // [H_q][d_h/8] swizzled
     const int64_t i = a.row0 + blockIdx.x;
     const int64_t prow = blockIdx.x;
-    const int n_sel = a.nsel ? a.nsel[prow] : (int)min((int64_t)a.k, i / a.local_of_row_div + 1);
+    const int64_t il = a.row_start ? i - a.row_start[i] : i; // row index within its sequence
+    const int n_sel = a.nsel ? a.nsel[prow] : (int)min((int64_t)a.k, il / a.local_of_row_div + 1);
     if (n_sel <= 0) return; // rejected decode sequence: output left unwritten
     const float* lp = a.lse_part + prow * a.k * a.H_q;
     for (int h = threadIdx.x; h < a.H_q; h += blockDim.x) {

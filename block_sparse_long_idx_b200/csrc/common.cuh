@@ -47,6 +47,10 @@ struct IndexTopkArgs {
     int H_kv, d_idx, k;
     int32_t* block_idx;
     int* err;
+    // packed batch of sequences (nullptr: one sequence of N rows): items are (sequence, tile pair)
+    const int2* vitems = nullptr; // [n_vitems] (sequence, pair u), decreasing work first
+    int n_vitems = 0;
+    const int32_t* cu = nullptr; // [B+1] first row of each sequence
 };
 cudaError_t launch_index_topk(const IndexTopkArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                               cudaStream_t s);
@@ -64,6 +68,9 @@ struct Kv2qArgs {
     int64_t max_items;
     int32_t* scan_tmp;
     int* err;
+    // packed batch (nullptr: one sequence): selections hold blocks local to the row's sequence
+    const int32_t* row_start = nullptr; // [N] first row of the row's sequence
+    const int32_t* row_gb0 = nullptr;   // [N] global index of the row's sequence's block 0
 };
 cudaError_t launch_kv2q(const Kv2qArgs& a, cudaStream_t s);
 size_t kv2q_scan_tmp_bytes(int64_t n, int H_kv);
@@ -78,6 +85,7 @@ struct AttnArgs {
     int64_t row0;               // first row of the pass (= w0 * window)
     int64_t rows_pass;          // rows the partial buffers hold
     int* item_counter;          // work items claimed so far in this launch (zero at launch)
+    const int32_t* blk_tok = nullptr; // packed batch: first row of each global block (nullptr: b * B_k)
     long long* timeline;        // optional: CTA 0 records clock64 per tile event (nullptr = off)
     int timeline_tiles;         // capacity in tiles (16 event slots per tile)
     uint16_t* o_part;           // [rows][k][H_q][d_h]
@@ -99,8 +107,14 @@ struct CombineArgs {
     const int32_t* nsel;      // optional per-row count of valid slots (decode), else NULL
     uint16_t* out;            // [*, H_q, d_h] rows offset by row0
     float* lse;               // nullable
+    const int32_t* row_start = nullptr; // packed batch: first row of each row's sequence (local index)
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+// Packed batch tables from cu[B+1] and blk_base[B+1] (global block of each sequence's block 0):
+// row_start[i], row_gb0[i] for every row, blk_tok[gb] for every global block.
+cudaError_t launch_varlen_tables(const int32_t* cu, const int32_t* blk_base, int B, int64_t T, int32_t nb_total,
+                                 int32_t* row_start, int32_t* row_gb0, int32_t* blk_tok, cudaStream_t s);
 
 struct DecodeArgs {
     const uint16_t* q;

@@ -42,13 +42,32 @@ struct IdxShared {
     int abort_flag;
 };
 
-__device__ __forceinline__ void item_of(int j, int n_pairs, int H_kv, int n_qt, int& r, int& u, bool& tb_valid,
-                                        int& steps)
+// Work item j: group r = j % H_kv and a pair u of query tiles (2u, 2u+1) of one sequence, whose
+// rows are [row0, row0 + nrows) of the packed tensors (one sequence of N rows unless a.vitems).
+struct IdxItem {
+    int r, u, steps;
+    bool tbv;
+    int row0, nrows;
+};
+
+__device__ __forceinline__ IdxItem item_at(const IndexTopkArgs& a, int j, int n_pairs)
 {
-    u = n_pairs - 1 - j / H_kv;
-    r = j % H_kv;
-    tb_valid = (2 * u + 1) < n_qt;
-    steps = tb_valid ? 2 * u + 1 : 2 * u;
+    IdxItem it;
+    it.r = j % a.H_kv;
+    if (a.vitems) {
+        const int2 v = a.vitems[j / a.H_kv];
+        it.u = v.y;
+        it.row0 = a.cu[v.x];
+        it.nrows = a.cu[v.x + 1] - it.row0;
+    } else {
+        it.u = n_pairs - 1 - j / a.H_kv;
+        it.row0 = 0;
+        it.nrows = (int)a.N;
+    }
+    const int n_qt = (it.nrows + kBk - 1) / kBk;
+    it.tbv = (2 * it.u + 1) < n_qt;
+    it.steps = it.tbv ? 2 * it.u + 1 : 2 * it.u;
+    return it;
 }
 
 __device__ __forceinline__ int item_for_round(int round, int cta, int P)
@@ -71,7 +90,7 @@ __global__ void __launch_bounds__(384, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_qt = (int)((a.N + kBk - 1) / kBk);
     const int n_pairs = (n_qt + 1) / 2;
-    const int n_items = n_pairs * a.H_kv;
+    const int n_items = (a.vitems ? a.n_vitems : n_pairs) * a.H_kv;
     const int P = gridDim.x, cta = blockIdx.x;
     volatile int* abort_flag = &sh.abort_flag;
 
@@ -107,16 +126,17 @@ __global__ void __launch_bounds__(384, 1)
             for (int round = 0; ok; ++round) {
                 const int j = item_for_round(round, cta, P);
                 if (j >= n_items) break;
-                int r, u, steps;
-                bool tbv;
-                item_of(j, n_pairs, a.H_kv, n_qt, r, u, tbv, steps);
+                const IdxItem itm = item_at(a, j, n_pairs);
+                const int r = itm.r, u = itm.u, steps = itm.steps;
+                const bool tbv = itm.tbv;
                 if (!wait_or_abort(&sh.q_empty, (item_cnt & 1) ^ 1, abort_flag, a.err, 1, kWaitLimit)) break;
                 mbar_arrive_expect_tx(&sh.q_full, C::TILE_BYTES * (tbv ? 2 : 1));
                 for (int c = 0; c < C::NKC; ++c) {
-                    tma_load_3d(sqA + c * C::CHUNK_BYTES, &qmap, &sh.q_full, c * C::CHUNK_COLS, r, 2 * u * kBk);
+                    tma_load_3d(sqA + c * C::CHUNK_BYTES, &qmap, &sh.q_full, c * C::CHUNK_COLS, r,
+                                itm.row0 + 2 * u * kBk);
                     if (tbv)
                         tma_load_3d(sqB + c * C::CHUNK_BYTES, &qmap, &sh.q_full, c * C::CHUNK_COLS, r,
-                                    (2 * u + 1) * kBk);
+                                    itm.row0 + (2 * u + 1) * kBk);
                 }
                 for (int b = 0; b < steps; ++b, ++gstep) {
                     const int s = gstep % C::NST;
@@ -127,7 +147,7 @@ __global__ void __launch_bounds__(384, 1)
                     mbar_arrive_expect_tx(&sh.kv_full[s], C::TILE_BYTES);
                     for (int c = 0; c < C::NKC; ++c)
                         tma_load_3d(sk + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &kmap, &sh.kv_full[s],
-                                    c * C::CHUNK_COLS, r, b * kBk);
+                                    c * C::CHUNK_COLS, r, itm.row0 + b * kBk);
                 }
                 ++item_cnt;
             }
@@ -146,9 +166,9 @@ __global__ void __launch_bounds__(384, 1)
             for (int round = 0; ok; ++round) {
                 const int j = item_for_round(round, cta, P);
                 if (j >= n_items) break;
-                int r, u, steps;
-                bool tbv;
-                item_of(j, n_pairs, a.H_kv, n_qt, r, u, tbv, steps);
+                const IdxItem itm = item_at(a, j, n_pairs);
+                const int u = itm.u, steps = itm.steps;
+                const bool tbv = itm.tbv;
                 if (!poll_or_abort(&sh.q_full, item_cnt & 1, abort_flag, a.err, 3, kWaitLimit)) break;
                 tc_fence_after();
                 for (int b = 0; b < steps; ++b, ++gstep, ++acc_cnt) {
@@ -187,9 +207,9 @@ __global__ void __launch_bounds__(384, 1)
         for (int round = 0;; ++round) {
             const int j = item_for_round(round, cta, P);
             if (j >= n_items) break;
-            int r, u, steps;
-            bool tbv;
-            item_of(j, n_pairs, a.H_kv, n_qt, r, u, tbv, steps);
+            const IdxItem itm = item_at(a, j, n_pairs);
+            const int r = itm.r, u = itm.u, steps = itm.steps;
+            const bool tbv = itm.tbv;
             const int tile = 2 * u + e;
             const bool active = (e == 0) || tbv;
             TopkList list;
@@ -227,8 +247,9 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (!ok) break;
             if (active) {
-                const int64_t i = (int64_t)tile * kBk + row;
-                if (i < a.N) emit_selection(list, tile, a.k, a.block_idx + ((int64_t)r * a.N + i) * a.k);
+                const int il = tile * kBk + row; // row within its sequence
+                if (il < itm.nrows)
+                    emit_selection(list, tile, a.k, a.block_idx + ((int64_t)r * a.N + itm.row0 + il) * a.k);
             }
         }
     }
@@ -250,7 +271,7 @@ cudaError_t launch_dk(const IndexTopkArgs& a, const CUtensorMap& qmap, const CUt
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     const int n_qt = (int)((a.N + kBk - 1) / kBk);
-    const int n_items = ((n_qt + 1) / 2) * a.H_kv;
+    const int n_items = (a.vitems ? a.n_vitems : (n_qt + 1) / 2) * a.H_kv;
     const int grid = n_items < n_sm ? n_items : n_sm;
     index_topk_kernel<DK><<<grid, 384, C::SMEM + sizeof(IdxShared), s>>>(a, qmap, kmap);
     note_launch(1);

@@ -29,10 +29,13 @@ __global__ void kv2q_count_kernel(Kv2qArgs a)
     const int64_t row_hi = min(a.N, row_lo + a.window);
     const int32_t* sel = a.block_idx + (int64_t)r * a.N * a.k;
     for (int64_t e = row_lo * a.k + threadIdx.x; e < row_hi * a.k; e += blockDim.x) {
-        const int32_t b = sel[e];
+        int32_t b = sel[e];
         const int64_t i = e / a.k;
         if (b < 0) continue;
-        if (b >= a.nb || (int64_t)b * kBk > i) {
+        // packed batch: the selection holds a block of the row's own sequence; key on its global index
+        const int64_t il = a.row_start ? i - a.row_start[i] : i;
+        if (a.row_gb0) b += a.row_gb0[i];
+        if (b >= a.nb || (int64_t)(b - (a.row_gb0 ? a.row_gb0[i] : 0)) * kBk > il) {
             report_error(a.err, MSA_ERR_DEVICE_CHECK, 100);
             continue;
         }
@@ -200,7 +203,11 @@ __global__ void kv2q_scatter_kernel(Kv2qArgs a)
         for (int u = 0; u < kAhead; ++u) {
             const int64_t i = i00 + (int64_t)u * rows_per_step + lane / a.k;
             int32_t b = bs[u];
-            if (b >= a.nb || (b >= 0 && (int64_t)b * kBk > i)) b = -1; // reported by the count pass
+            if (b >= 0) {
+                const int64_t il = a.row_start ? i - a.row_start[i] : i;
+                const int32_t g0 = a.row_gb0 ? a.row_gb0[i] : 0;
+                b = (b + g0 >= a.nb || (int64_t)b * kBk > il) ? -1 : b + g0; // invalid ones: reported by the count pass
+            }
             const unsigned peers = __match_any_sync(0xffffffffu, b);
             if (b >= 0) {
                 const unsigned before = peers & lt_mask;

@@ -5,6 +5,9 @@
 #include <cstring>
 #include <mutex>
 
+#include <algorithm>
+#include <vector>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -187,10 +190,15 @@ msa_status msa_index_topk(const msa_bf16* q_idx, const msa_bf16* k_idx, int64_t 
 }
 
 // ------------------------------------------------------------------------------------ kv2q
-msa_status msa_kv2q_layout_get(int64_t N, int H_kv, int B_k, int k, int window, int chunk, msa_kv2q_layout* L)
+} // extern "C"
+
+// Layout of an inversion over N rows whose selections name nb distinct blocks (nb = ceil(N / B_k)
+// for one sequence; the sum of the sequences' block counts for a packed batch).
+static msa_status layout_fill(int64_t N, int H_kv, int B_k, int k, int64_t nb, int window, int chunk,
+                              msa_kv2q_layout* L)
 {
-    if (!L || N < 1 || H_kv < 1 || B_k < 1 || k < 1 || window < 0 || chunk < 0) return MSA_ERR_INVALID_ARG;
-    if (B_k != kBk || k > kMaxK || N > kMaxN) return MSA_ERR_UNSUPPORTED;
+    if (!L || N < 1 || H_kv < 1 || B_k < 1 || k < 1 || window < 0 || chunk < 0 || nb < 1) return MSA_ERR_INVALID_ARG;
+    if (B_k != kBk || k > kMaxK || N > kMaxN || nb > (int64_t)kMaxN) return MSA_ERR_UNSUPPORTED;
     if (window == 0) window = kDefaultWindow;
     if (chunk == 0) chunk = kDefaultChunk < window ? kDefaultChunk : window;
     if (window % kBk != 0 || chunk > window) return MSA_ERR_INVALID_ARG;
@@ -199,14 +207,15 @@ msa_status msa_kv2q_layout_get(int64_t N, int H_kv, int B_k, int k, int window, 
     L->H_kv = H_kv;
     L->B_k = B_k;
     L->k = k;
-    L->nb = (int32_t)((N + B_k - 1) / B_k);
+    L->nb = (int32_t)nb;
     L->window = window;
     L->chunk = chunk;
     L->n_windows = (int32_t)((N + window - 1) / window);
     int64_t max_items = 0;
     for (int64_t w = 0; w < L->n_windows; ++w) {
         const int64_t lo = w * window, hi = (w + 1) * window < N ? (w + 1) * window : N;
-        const int64_t vis = (hi - 1) / B_k + 1;
+        const int64_t vis_one = (hi - 1) / B_k + 1; // blocks visible to the window's rows (one sequence)
+        const int64_t vis = vis_one < nb ? vis_one : nb;
         max_items += (int64_t)H_kv * (vis + ((hi - lo) * k + chunk - 1) / chunk);
     }
     L->max_items = max_items;
@@ -228,13 +237,22 @@ msa_status msa_kv2q_layout_get(int64_t N, int H_kv, int B_k, int k, int window, 
     return MSA_OK;
 }
 
+extern "C" {
+
+msa_status msa_kv2q_layout_get(int64_t N, int H_kv, int B_k, int k, int window, int chunk, msa_kv2q_layout* L)
+{
+    if (!L || N < 1 || B_k < 1) return MSA_ERR_INVALID_ARG;
+    return layout_fill(N, H_kv, B_k, k, (N + B_k - 1) / B_k, window, chunk, L);
+}
+
 size_t msa_build_kv2q_workspace_size(const msa_kv2q_layout* L)
 {
     return L ? kErrBytes + kv2q_internal_tmp(*L) : 0;
 }
 
 static msa_status build_kv2q_impl(const int32_t* block_idx, const msa_kv2q_layout* L, void* kv2q, int* err,
-                                  void* tmp, cudaStream_t s)
+                                  void* tmp, cudaStream_t s, const int32_t* row_start = nullptr,
+                                  const int32_t* row_gb0 = nullptr)
 {
     uint8_t* base = (uint8_t*)kv2q;
     Kv2qArgs a;
@@ -255,6 +273,8 @@ static msa_status build_kv2q_impl(const int32_t* block_idx, const msa_kv2q_layou
     a.max_items = L->max_items;
     a.scan_tmp = (int32_t*)tmp;
     a.err = err;
+    a.row_start = row_start;
+    a.row_gb0 = row_gb0;
     trace_begin(s);
     const cudaError_t e = launch_kv2q(a, s);
     trace_end(s, MSA_KERNEL_KV2Q);
@@ -286,6 +306,62 @@ msa_status msa_build_kv2q(const int32_t* block_idx, const msa_kv2q_layout* L, vo
 
 // ------------------------------------------------------------------------------------ sparse prefill
 static size_t partial_row_bytes(int H_q, int d_h, int k) { return (size_t)k * H_q * ((size_t)d_h * 2 + 4); }
+
+// Attention + combine over the windows of an inversion, wins_per_pass windows per pass.
+static msa_status run_passes(const uint8_t* kvb, const msa_kv2q_layout* L, int64_t N, int H_q, int H_kv, int d_h, int k,
+                             const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                             int64_t wins_per_pass, int64_t rows_pass, uint16_t* o_part, float* lse_part,
+                             msa_bf16* out, float* lse, void* workspace, cudaStream_t s, const int32_t* blk_tok,
+                             const int32_t* row_start)
+{
+    for (int64_t w0 = 0; w0 < L->n_windows; w0 += wins_per_pass) {
+        const int64_t w1 = w0 + wins_per_pass < L->n_windows ? w0 + wins_per_pass : L->n_windows;
+        AttnArgs a;
+        a.N = N;
+        a.H_q = H_q;
+        a.H_kv = H_kv;
+        a.d_h = d_h;
+        a.k = k;
+        a.entries = (const int32_t*)(kvb + L->entries);
+        a.items = (const msa_work_item*)(kvb + L->items);
+        a.window_items = (const int32_t*)(kvb + L->window_items);
+        a.w0 = (int)w0;
+        a.w1 = (int)w1;
+        a.row0 = w0 * L->window;
+        a.rows_pass = rows_pass;
+        a.item_counter = (int*)workspace + 4; // inside the error-word region, reset for every pass
+        a.blk_tok = blk_tok;
+        a.timeline = nullptr;
+        a.timeline_tiles = 0;
+        a.o_part = o_part;
+        a.lse_part = lse_part;
+        a.err = (int*)workspace;
+        if (msa_status st1 = cuda_status(cudaMemsetAsync(a.item_counter, 0, sizeof(int), s), "clearing the work counter"))
+            return st1;
+        trace_begin(s);
+        const cudaError_t ea = launch_sparse_attn(a, qmap, kmap, vmap, s);
+        trace_end(s, MSA_KERNEL_ATTN);
+        if (ea != cudaSuccess) return cuda_status(ea, "attention launch");
+        CombineArgs c;
+        c.row0 = a.row0;
+        c.n_rows = (w1 * L->window < N ? w1 * L->window : N) - a.row0;
+        c.H_q = H_q;
+        c.d_h = d_h;
+        c.k = k;
+        c.local_of_row_div = kBk;
+        c.o_part = o_part;
+        c.lse_part = lse_part;
+        c.nsel = nullptr;
+        c.out = out;
+        c.lse = lse;
+        c.row_start = row_start;
+        trace_begin(s);
+        const cudaError_t ec = launch_combine(c, s);
+        trace_end(s, MSA_KERNEL_COMBINE);
+        if (ec != cudaSuccess) return cuda_status(ec, "combine launch");
+    }
+    return MSA_OK;
+}
 
 size_t msa_sparse_prefill_workspace_size(int64_t N, int H_q, int H_kv, int d_h, int B_k, int k,
                                          int64_t max_rows_per_pass, int internal_kv2q)
@@ -360,52 +436,182 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
         msa_status st = build_kv2q_impl(block_idx, L, kvbuf, (int*)workspace, kvtmp, s);
         if (st != MSA_OK) return st;
     }
-    const uint8_t* kvb = (const uint8_t*)kv;
-    for (int64_t w0 = 0; w0 < L->n_windows; w0 += wins_per_pass) {
-        const int64_t w1 = w0 + wins_per_pass < L->n_windows ? w0 + wins_per_pass : L->n_windows;
-        AttnArgs a;
-        a.N = N;
-        a.H_q = H_q;
-        a.H_kv = H_kv;
-        a.d_h = d_h;
-        a.k = k;
-        a.entries = (const int32_t*)(kvb + L->entries);
-        a.items = (const msa_work_item*)(kvb + L->items);
-        a.window_items = (const int32_t*)(kvb + L->window_items);
-        a.w0 = (int)w0;
-        a.w1 = (int)w1;
-        a.row0 = w0 * L->window;
-        a.rows_pass = rows_pass;
-        a.item_counter = (int*)workspace + 4; // inside the error-word region, reset for every pass
-        a.timeline = nullptr;
-        a.timeline_tiles = 0;
-        a.o_part = o_part;
-        a.lse_part = lse_part;
-        a.err = (int*)workspace;
-        if (msa_status st1 = cuda_status(cudaMemsetAsync(a.item_counter, 0, sizeof(int), s), "clearing the work counter"))
-            return st1;
-        trace_begin(s);
-        const cudaError_t ea = launch_sparse_attn(a, qmap, kmap, vmap, s);
-        trace_end(s, MSA_KERNEL_ATTN);
-        if (ea != cudaSuccess) return cuda_status(ea, "attention launch");
-        CombineArgs c;
-        c.row0 = a.row0;
-        c.n_rows = (w1 * L->window < N ? w1 * L->window : N) - a.row0;
-        c.H_q = H_q;
-        c.d_h = d_h;
-        c.k = k;
-        c.local_of_row_div = kBk;
-        c.o_part = o_part;
-        c.lse_part = lse_part;
-        c.nsel = nullptr;
-        c.out = out;
-        c.lse = lse;
-        trace_begin(s);
-        const cudaError_t ec = launch_combine(c, s);
-        trace_end(s, MSA_KERNEL_COMBINE);
-        if (ec != cudaSuccess) return cuda_status(ec, "combine launch");
+    return run_passes((const uint8_t*)kv, L, N, H_q, H_kv, d_h, k, qmap, kmap, vmap, wins_per_pass, rows_pass, o_part,
+                      lse_part, out, lse, workspace, s, nullptr, nullptr);
+}
+
+// ------------------------------------------------------------------------------------ varlen prefill
+} // extern "C"
+
+namespace {
+
+// Host-side plan of a packed batch: global block bases and the index work items (sequence, tile
+// pair) in decreasing work order.
+struct VarlenPlan {
+    int B = 0;
+    int64_t T = 0, NB = 0;
+    std::vector<int32_t> head; // [cu (B+1) | blk_base (B+1) | vitems (2 * n_vitems)], copied to the device
+    int n_vitems = 0;
+    size_t off_cu = 0, off_base = 0, off_items = 0, head_bytes = 0;
+};
+
+msa_status varlen_plan(const int32_t* cu, int B, VarlenPlan& p)
+{
+    if (!cu || B < 1 || cu[0] != 0) return MSA_ERR_INVALID_ARG;
+    for (int s = 0; s < B; ++s)
+        if (cu[s + 1] < cu[s]) return MSA_ERR_INVALID_ARG;
+    p.B = B;
+    p.T = cu[B];
+    if (p.T < 1) return MSA_ERR_INVALID_ARG;
+    if (p.T > kMaxN) return MSA_ERR_UNSUPPORTED;
+    std::vector<int32_t> base(B + 1, 0);
+    std::vector<std::pair<int, int>> items; // (u, s)
+    for (int s = 0; s < B; ++s) {
+        const int n_qt = (cu[s + 1] - cu[s] + kBk - 1) / kBk;
+        base[s + 1] = base[s] + n_qt;
+        for (int u = 0; u < (n_qt + 1) / 2; ++u) items.emplace_back(u, s);
+    }
+    p.NB = base[B];
+    std::stable_sort(items.begin(), items.end(), [](const std::pair<int, int>& x, const std::pair<int, int>& y) {
+        return x.first > y.first; // most work first
+    });
+    p.n_vitems = (int)items.size();
+    p.off_cu = 0;
+    p.off_base = align_up((size_t)(B + 1) * 4, 16);
+    p.off_items = p.off_base + align_up((size_t)(B + 1) * 4, 16);
+    p.head_bytes = align_up(p.off_items + (size_t)p.n_vitems * 8, 256);
+    p.head.assign(p.head_bytes / 4, 0);
+    for (int s = 0; s <= B; ++s) {
+        p.head[p.off_cu / 4 + s] = cu[s];
+        p.head[p.off_base / 4 + s] = base[s];
+    }
+    for (int j = 0; j < p.n_vitems; ++j) {
+        p.head[p.off_items / 4 + 2 * j] = items[j].second;
+        p.head[p.off_items / 4 + 2 * j + 1] = items[j].first;
     }
     return MSA_OK;
+}
+
+// Workspace carve-up of msa_sparse_prefill_varlen; rows_pass = 0 in the plan means "size query".
+struct VarlenWs {
+    size_t head, row_start, row_gb0, blk_tok, kv2q, kvtmp, parts, total;
+    int64_t rows_pass;
+    msa_kv2q_layout L;
+};
+
+msa_status varlen_ws(const VarlenPlan& p, int H_q, int H_kv, int d_h, int k, int64_t max_rows_per_pass,
+                     size_t workspace_bytes, VarlenWs& w)
+{
+    if (msa_status st = layout_fill(p.T, H_kv, kBk, k, p.NB, 0, 0, &w.L)) return st;
+    size_t off = kErrBytes;
+    w.head = off;
+    off += p.head_bytes;
+    w.row_start = off;
+    off += align_up((size_t)p.T * 4, 256);
+    w.row_gb0 = off;
+    off += align_up((size_t)p.T * 4, 256);
+    w.blk_tok = off;
+    off += align_up((size_t)p.NB * 4, 256);
+    w.kv2q = off;
+    off += align_up(w.L.total_bytes, 256);
+    w.kvtmp = off;
+    off += align_up(kv2q_internal_tmp(w.L), 256);
+    w.parts = off;
+    const size_t per_row = partial_row_bytes(H_q, d_h, k);
+    if (workspace_bytes == 0) { // size query: room for max_rows_per_pass rows (whole windows)
+        int64_t rows = max_rows_per_pass <= 0 || max_rows_per_pass > p.T ? p.T : max_rows_per_pass;
+        rows = (rows + w.L.window - 1) / w.L.window * w.L.window;
+        w.rows_pass = rows;
+        w.total = off + 512 + align_up((size_t)rows * k * H_q * d_h * 2, 256) + align_up((size_t)rows * k * H_q * 4, 256);
+        return MSA_OK;
+    }
+    if (workspace_bytes <= off + 512) return MSA_ERR_WORKSPACE;
+    const int64_t wins = (int64_t)((workspace_bytes - off - 512) / per_row) / w.L.window;
+    if (wins < 1) return MSA_ERR_WORKSPACE;
+    w.rows_pass = (wins < w.L.n_windows ? wins : w.L.n_windows) * w.L.window;
+    w.total = workspace_bytes;
+    return MSA_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+size_t msa_sparse_prefill_varlen_workspace_size(const int32_t* cu_seqlens, int B, int H_q, int H_kv, int d_h, int B_k,
+                                                int k, int64_t max_rows_per_pass)
+{
+    VarlenPlan p;
+    VarlenWs w;
+    if (B_k != kBk || H_q < 1 || H_kv < 1 || d_h < 1 || varlen_plan(cu_seqlens, B, p) != MSA_OK ||
+        varlen_ws(p, H_q, H_kv, d_h, k, max_rows_per_pass, 0, w) != MSA_OK)
+        return 0;
+    return w.total;
+}
+
+msa_status msa_sparse_prefill_varlen(const msa_bf16* q, const msa_bf16* kk, const msa_bf16* v, const msa_bf16* q_idx,
+                                     const msa_bf16* k_idx, const int32_t* cu_seqlens, int B, int H_q, int H_kv,
+                                     int d_h, int d_idx, int B_k, int k, int32_t* block_idx, msa_bf16* out, float* lse,
+                                     void* workspace, size_t workspace_bytes, msa_stream_t stream)
+{
+    if (!q || !kk || !v || !q_idx || !k_idx || !block_idx || !out || !workspace || H_q < 1 || H_kv < 1 || d_h < 1 ||
+        d_idx < 1 || k < 1 || H_q % H_kv != 0)
+        return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(kk, 16) || !aligned(v, 16) || !aligned(q_idx, 16) || !aligned(k_idx, 16) ||
+        !aligned(block_idx, 4) || !aligned(out, 16) || !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+        return MSA_ERR_INVALID_ARG;
+    const int G = H_q / H_kv;
+    if (B_k != kBk || k > kMaxK || !(d_h == 64 || d_h == 128) || !pow2(G) || G > 128 ||
+        !(d_idx == 32 || d_idx == 64 || d_idx == 128) || H_kv > 65535)
+        return MSA_ERR_UNSUPPORTED;
+    VarlenPlan p;
+    if (msa_status st = varlen_plan(cu_seqlens, B, p)) return st;
+    VarlenWs w;
+    if (msa_status st = varlen_ws(p, H_q, H_kv, d_h, k, 0, workspace_bytes, w)) return st;
+    if (injected("msa_sparse_prefill_varlen")) return MSA_ERR_CUDA;
+    const int64_t T = p.T;
+    CUtensorMap qim, kim, qmap, kmap, vmap;
+    const uint32_t box0 = d_idx < 64 ? (uint32_t)d_idx : 64u;
+    const CUtensorMapSwizzle sw = d_idx == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_map_3d(&qim, q_idx, d_idx, H_kv, T, box0, 1, kBk, sw) ||
+        !make_map_3d(&kim, k_idx, d_idx, H_kv, T, box0, 1, kBk, sw) ||
+        !make_map_3d(&qmap, q, d_h, H_q, T, 64, G, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d(&kmap, kk, d_h, H_kv, T, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d(&vmap, v, d_h, H_kv, T, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B))
+        return MSA_ERR_INVALID_ARG;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* ws = (uint8_t*)workspace;
+    const int32_t* d_cu = (const int32_t*)(ws + w.head + p.off_cu);
+    const int32_t* d_base = (const int32_t*)(ws + w.head + p.off_base);
+    const int2* d_items = (const int2*)(ws + w.head + p.off_items);
+    int32_t* row_start = (int32_t*)(ws + w.row_start);
+    int32_t* row_gb0 = (int32_t*)(ws + w.row_gb0);
+    int32_t* blk_tok = (int32_t*)(ws + w.blk_tok);
+    if (msa_status st = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st;
+    if (msa_status st = cuda_status(cudaMemcpyAsync(ws + w.head, p.head.data(), p.head_bytes, cudaMemcpyHostToDevice, s),
+                                    "copying the batch plan"))
+        return st;
+    if (msa_status st = cuda_status(launch_varlen_tables(d_cu, d_base, B, T, (int32_t)p.NB, row_start, row_gb0, blk_tok, s),
+                                    "varlen tables launch"))
+        return st;
+    // index branch over (sequence, tile pair) items
+    IndexTopkArgs ia{q_idx, k_idx, T, H_kv, d_idx, k, block_idx, (int*)workspace};
+    ia.vitems = d_items;
+    ia.n_vitems = p.n_vitems;
+    ia.cu = d_cu;
+    trace_begin(s);
+    const cudaError_t ei = launch_index_topk(ia, qim, kim, s);
+    trace_end(s, MSA_KERNEL_INDEX_TOPK);
+    if (ei != cudaSuccess) return cuda_status(ei, "index_topk launch");
+    // inversion keyed on global blocks
+    if (msa_status st = build_kv2q_impl(block_idx, &w.L, ws + w.kv2q, (int*)workspace, ws + w.kvtmp, s, row_start,
+                                        row_gb0))
+        return st;
+    const int64_t wins_per_pass = w.rows_pass / w.L.window;
+    uint16_t* o_part = (uint16_t*)(ws + w.parts);
+    float* lse_part = (float*)(ws + w.parts + align_up((size_t)w.rows_pass * k * H_q * d_h * 2, 256));
+    return run_passes(ws + w.kv2q, &w.L, T, H_q, H_kv, d_h, k, qmap, kmap, vmap, wins_per_pass, w.rows_pass, o_part,
+                      lse_part, out, lse, workspace, s, blk_tok, row_start);
 }
 
 // ------------------------------------------------------------------------------------ decode

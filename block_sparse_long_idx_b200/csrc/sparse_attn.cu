@@ -59,6 +59,7 @@ struct TileRec {
     int32_t r, b;  // GQA group, KV block
     int32_t npos;  // positions in the tile (1 .. 128/G); -1 marks the end of the CTA's work
     int32_t flags; // bit 0: first tile of its item, bit 1: last tile, bit 2: K/V stage of the item
+    int32_t tok0;  // first row of block b (b * 128, or from the block table of a packed batch)
 };
 
 struct AttnShared {
@@ -168,12 +169,11 @@ __global__ void __launch_bounds__(512, 1)
                     const int s = it & 1;
                     if (!wait_or_abort(&sh.kv_empty[s], ((it >> 1) & 1) ^ 1, abort_flag, a.err, 20, kWaitLimit))
                         break;
+                    const int tok0 = a.blk_tok ? a.blk_tok[item.b] : item.b * kBk;
                     mbar_arrive_expect_tx(&sh.kv_full[s], 2 * C::TILE);
                     for (int c = 0; c < C::NKC; ++c) {
-                        tma_load_3d(sK + s * C::TILE + c * C::CHUNK, &kmap, &sh.kv_full[s], c * 64, item.r,
-                                    item.b * kBk);
-                        tma_load_3d(sV + s * C::TILE + c * C::CHUNK, &vmap, &sh.kv_full[s], c * 64, item.r,
-                                    item.b * kBk);
+                        tma_load_3d(sK + s * C::TILE + c * C::CHUNK, &kmap, &sh.kv_full[s], c * 64, item.r, tok0);
+                        tma_load_3d(sV + s * C::TILE + c * C::CHUNK, &vmap, &sh.kv_full[s], c * 64, item.r, tok0);
                     }
                 }
                 for (int g = it - 1; g >= 0 && g >= it - 2; --g)
@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(512, 1)
                 if (!ok) break;
                 const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
                 const int ntiles = (item.len + PPT - 1) / PPT;
+                const int tok0 = a.blk_tok ? a.blk_tok[item.b] : item.b * kBk;
                 for (int t = 0; t < ntiles; ++t, ++qt) {
                     const int qs = qt % NQ, rs = qt % kRing;
                     const int npos = min(PPT, item.len - t * PPT);
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     if (lane == 0)
                         sh.rec[rs] = TileRec{item.r, item.b, npos,
-                                             (t == 0 ? 1 : 0) | (t == ntiles - 1 ? 2 : 0) | ((it & 1) << 2)};
+                                             (t == 0 ? 1 : 0) | (t == ntiles - 1 ? 2 : 0) | ((it & 1) << 2), tok0};
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh.tile_full[rs]);
                     if (lane == 0)
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(512, 1)
                     if (qt >= kRing && !wait_or_abort(&sh.tile_free[rs], ((qt / kRing) & 1) ^ 1, abort_flag, a.err,
                                                       33, kWaitLimit))
                         break;
-                    sh.rec[rs] = TileRec{0, 0, -1, 0};
+                    sh.rec[rs] = TileRec{0, 0, -1, 0, 0};
                     mbar_arrive(&sh.tile_full[rs]);
                 }
             }
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(512, 1)
             const TileRec rec = sh.rec[rs];
             if (rec.npos < 0) break;
             const int qa = qt & 1;
-            const int limit = pl < rec.npos ? min(127, sh.rec_e[rs][pl] / a.k - rec.b * kBk) : 127;
+            const int limit = pl < rec.npos ? min(127, sh.rec_e[rs][pl] / a.k - rec.tok0) : 127;
             if (!wait_or_abort(&sh.s_full[qa], (qt >> 1) & 1, abort_flag, a.err, 26, kWaitLimit)) break;
             if (row == 0) TL(4, qt);
             tc_fence_after();

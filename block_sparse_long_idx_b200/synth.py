@@ -169,6 +169,45 @@ DECODE64 = DecodeConfig("decode_B64_L16K-128K", B=64, L_max=131072, len_lo=16384
 DECODE64_SHORT = DecodeConfig("decode_B64_L2K-16K", B=64, L_max=16384, len_lo=2048, len_hi=16384, H_q=64, H_kv=4,
                               d_h=128, d_idx=64, B_k=128, k=16, seed=5)
 
+@dataclass(frozen=True)
+class VarlenConfig:
+    """A batch of independent causal sequences packed along the token axis (cu_seqlens layout)."""
+    name: str
+    lens: tuple
+    H_q: int
+    H_kv: int
+    d_h: int
+    d_idx: int
+    B_k: int
+    k: int
+    seed: int
+
+    @property
+    def T(self) -> int:
+        return int(sum(self.lens))
+
+    def cu_seqlens(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.lens)]).astype(np.int32)
+
+    def packed(self) -> "PrefillConfig":
+        return PrefillConfig(self.name, N=self.T, H_q=self.H_q, H_kv=self.H_kv, d_h=self.d_h, d_idx=self.d_idx,
+                             B_k=self.B_k, k=self.k, seed=self.seed)
+
+
+def varlen_lengths(n_seq: int, total: int, lo: int, seed: int) -> tuple:
+    """n_seq lengths >= lo summing to total, drawn from a seeded Dirichlet-like split (long/short mix)."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 77]))
+    w = rng.exponential(1.0, n_seq)
+    extra = total - n_seq * lo
+    lens = lo + np.floor(w / w.sum() * extra).astype(np.int64)
+    lens[: total - int(lens.sum())] += 1
+    return tuple(int(x) for x in lens)
+
+
+# 128K tokens as 16 sequences of mixed lengths (>= 1K): the serving-form prefill of the same model shape
+VARLEN128K = VarlenConfig("varlen_16seq_T131072", lens=varlen_lengths(16, 131072, 1024, 6), H_q=64, H_kv=4, d_h=128,
+                          d_idx=64, B_k=128, k=16, seed=6)
+
 PREFILL_CONFIGS = {c.name: c for c in (TINY, P32K, P128K, P1M)}
 DECODE_CONFIGS = {c.name: c for c in (DECODE64, DECODE64_SHORT)}
 
@@ -221,6 +260,14 @@ def prefill_qkv(cfg: PrefillConfig) -> dict:
 def prefill_inputs(cfg: PrefillConfig) -> dict:
     d = prefill_index_inputs(cfg)
     d.update(prefill_qkv(cfg))
+    return d
+
+
+def varlen_inputs(cfg: VarlenConfig) -> dict:
+    """Packed tensors of all sequences ([T, heads, dim], as prefill_inputs of one T-token sequence)
+    plus cu_seqlens [B+1] int32; every sequence is an independent causal problem."""
+    d = prefill_inputs(cfg.packed())
+    d["cu_seqlens"] = cfg.cu_seqlens()
     return d
 
 

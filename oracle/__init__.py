@@ -124,6 +124,27 @@ class Oracle:
         out, lse = self.attend_rows(inputs["q"], inputs["k"], inputs["v"], rows, sel, B_k, n_threads)
         return sel, out, lse
 
+    def prefill_varlen_rows(self, inputs: dict, cu_seqlens, rows, B_k: int, k: int, n_threads: int = 0):
+        """Packed batch of independent sequences (cu_seqlens [B+1]): each sequence is its own causal
+        problem, so each row is answered by the single-sequence path on its sequence's slice of the
+        packed tensors, in the sequence's local indices. Returns (sel [n, H_kv, k] with local block
+        ids, out, lse) for the given global rows."""
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        rows = np.asarray(rows, dtype=np.int64)
+        seq = np.searchsorted(cu, rows, side="right") - 1
+        H_kv = inputs["k_idx"].shape[1]
+        H_q, d_h = inputs["q"].shape[1], inputs["q"].shape[2]
+        sel = np.empty((len(rows), H_kv, k), dtype=np.int32)
+        out = np.empty((len(rows), H_q, d_h), dtype=np.float64)
+        lse = np.empty((len(rows), H_q), dtype=np.float64)
+        for s in np.unique(seq):
+            lo, hi = int(cu[s]), int(cu[s + 1])
+            pick = np.nonzero(seq == s)[0]
+            part = {n: np.ascontiguousarray(inputs[n][lo:hi]) for n in ("q", "k", "v", "q_idx", "k_idx")}
+            s_sel, s_out, s_lse = self.prefill_rows(part, rows[pick] - lo, B_k, k, n_threads)
+            sel[pick], out[pick], lse[pick] = s_sel, s_out, s_lse
+        return sel, out, lse
+
     def decode(self, inputs: dict, B_k: int, k: int, n_threads: int = 0):
         """Decode oracle. Returns (sel [B, H_kv, k], out f64 [B, H_q, d_h], lse f64 [B, H_q])."""
         q, qi = _u16(inputs["q"]), _u16(inputs["q_idx"])
@@ -171,6 +192,10 @@ def attend_rows(*a, **kw):
 
 def prefill_rows(*a, **kw):
     return default().prefill_rows(*a, **kw)
+
+
+def prefill_varlen_rows(*a, **kw):
+    return default().prefill_varlen_rows(*a, **kw)
 
 
 def decode(*a, **kw):

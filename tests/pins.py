@@ -248,6 +248,28 @@ def check_decode_matches_prefill_row(o):
         assert np.max(np.abs(lse[beta] - l2[0])) < 1e-13
 
 
+def check_varlen_matches_dense_per_sequence(o):
+    """A packed batch: each sequence's selection and attention equal the dense brute force run on that
+    sequence alone (tokens of other sequences are invisible, block indices restart at each sequence)."""
+    lens = [1, 5, 16, 37, 64, 130]
+    H_q, H_kv, d_h, d_idx, B_k, k = 4, 2, 8, 8, 16, 3
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T = int(cu[-1])
+    inp = _attn_inputs(T, H_q, H_kv, d_h, d_idx, 9)
+    rows = np.arange(T)
+    sel, out, lse = o.prefill_varlen_rows(inp, cu, rows, B_k, k)
+    for s in range(len(lens)):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        n = hi - lo
+        part = {name: inp[name][lo:hi] for name in inp}
+        want_sel = ref.dense_selection(part["q_idx"], part["k_idx"], B_k, k)
+        got_sel = np.ascontiguousarray(sel[lo:hi].transpose(1, 0, 2))
+        assert np.array_equal(got_sel, want_sel), s
+        want, want_lse = ref.masked_attention(part["q"], part["k"], part["v"], ref.selection_mask(want_sel, n, B_k))
+        assert np.max(np.abs(out[lo:hi] - want)) < 1e-12, s
+        assert np.max(np.abs(lse[lo:hi] - want_lse)) < 1e-12, s
+
+
 ALL_CHECKS = [
     check_selection_bruteforce,
     check_selection_ties_closed_form,
@@ -261,4 +283,5 @@ ALL_CHECKS = [
     check_combine_identity,
     check_kv2q_bruteforce,
     check_decode_matches_prefill_row,
+    check_varlen_matches_dense_per_sequence,
 ]

@@ -117,3 +117,31 @@ def test_selftest_validation(msa):
     assert lib.msa_selftest_wait_timeout(WS, 256, 0, None) == INVALID
     assert lib.msa_selftest_wait_timeout(WS, 256, 2_000_000_001, None) == INVALID
     assert lib.msa_selftest_wait_timeout(WS, 8, 1000, None) == WORKSPACE
+
+
+def test_varlen_validation_and_sizes(msa):
+    """Packed-batch prefill: cu_seqlens checks and workspace sizing happen on the host."""
+    lib = msa.lib
+    c_vp = ctypes.c_void_p
+    import numpy as np
+
+    def cu(*x):
+        a = np.asarray(x, dtype=np.int32)
+        return a, a.ctypes.data_as(c_vp)
+
+    good, gp = cu(0, 100, 100, 1000, 4096)
+    sz = lib.msa_sparse_prefill_varlen_workspace_size(gp, 4, 16, 2, 128, 128, 8, 0)
+    assert sz > 0
+    # fewer rows per pass -> smaller workspace, never below one window
+    assert 0 < lib.msa_sparse_prefill_varlen_workspace_size(gp, 4, 16, 2, 128, 128, 8, 2048) <= sz
+    for bad in ((1, 100), (0, 50, 40), (0, 0)):
+        b, bp = cu(*bad)
+        assert lib.msa_sparse_prefill_varlen_workspace_size(bp, len(bad) - 1, 16, 2, 128, 128, 8, 0) == 0
+        assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, bp, len(bad) - 1, 16, 2, 128, 64, 128, 8, P2, P, None, WS,
+                                             sz, None) == INVALID
+    args = (P, P, P, P, P, gp, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS)
+    assert lib.msa_sparse_prefill_varlen(*args, 256, None) == WORKSPACE
+    assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, gp, 4, 16, 2, 96, 64, 128, 8, P2, P, None, WS, sz,
+                                         None) == UNSUPPORTED
+    assert lib.msa_sparse_prefill_varlen(P + 8, P, P, P, P, gp, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS, sz,
+                                         None) == INVALID

@@ -1,0 +1,86 @@
+"""GPU parity, packed-batch (varlen) prefill: every sequence of a cu_seqlens batch is an independent
+causal problem. Selections (local block ids, bit-exact) and outputs (tolerance) against the oracle
+run on each sequence alone; ragged, tiny and empty sequences; several passes; and a batch of one
+sequence equal to the single-sequence entry points."""
+import zlib
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import block_sparse_long_idx_b200 as msa  # noqa: E402
+import oracle  # noqa: E402
+from block_sparse_long_idx_b200 import synth  # noqa: E402
+from tests.gpu_util import assert_lse_close, assert_out_close, assert_selection_equal, bf16_to_f64, dev  # noqa: E402
+
+# name, lengths, H_q, H_kv, d_h, d_idx, k, check all rows
+CASES = [
+    ("ragged_small", (1, 5, 127, 128, 129, 300, 1000, 2049), 8, 2, 64, 32, 4, True),
+    ("empty_seqs", (0, 500, 0, 0, 300, 1), 4, 1, 128, 64, 3, True),
+    ("G16_mixed", (3000, 700, 5000, 1, 2500), 64, 4, 128, 64, 16, False),
+    ("G1_k8", (900, 1300, 64), 2, 2, 64, 128, 8, True),
+]
+
+
+def _cfg(name, lens, H_q, H_kv, d_h, d_idx, k):
+    return synth.VarlenConfig(name, lens=tuple(lens), H_q=H_q, H_kv=H_kv, d_h=d_h, d_idx=d_idx, B_k=128, k=k,
+                              seed=zlib.crc32(name.encode()) % 1000)
+
+
+def _check(cfg, rows, max_rows_per_pass=0):
+    inp = synth.varlen_inputs(cfg)
+    t = {n: dev(inp[n]) for n in ("q", "k", "v", "q_idx", "k_idx")}
+    out, lse, bi = msa.msa_sparse_prefill_varlen(t["q"], t["k"], t["v"], t["q_idx"], t["k_idx"], inp["cu_seqlens"],
+                                                 128, cfg.k, max_rows_per_pass=max_rows_per_pass)
+    torch.cuda.synchronize()
+    sel, want, want_lse = oracle.prefill_varlen_rows(inp, inp["cu_seqlens"], rows, 128, cfg.k)
+    got_sel = bi.cpu().numpy()[:, rows, :]
+    assert_selection_equal(got_sel, np.ascontiguousarray(sel.transpose(1, 0, 2)), rows)
+    assert_out_close(bf16_to_f64(out)[rows], want)
+    assert_lse_close(lse.cpu().numpy()[rows].astype(np.float64), want_lse)
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_varlen_prefill(case):
+    name, lens, H_q, H_kv, d_h, d_idx, k, full = case
+    cfg = _cfg(name, lens, H_q, H_kv, d_h, d_idx, k)
+    if full:
+        rows = np.arange(cfg.T)
+    else:  # every sequence's first, last and block-boundary rows plus a uniform sample
+        cu = cfg.cu_seqlens()
+        fixed = set()
+        for s in range(len(lens)):
+            if lens[s]:
+                for r in (0, 127, 128, lens[s] - 1):
+                    if r < lens[s]:
+                        fixed.add(int(cu[s]) + r)
+        rng = np.random.default_rng(5)
+        rows = np.unique(np.concatenate([np.array(sorted(fixed)), rng.choice(cfg.T, 400, replace=False)]))
+    _check(cfg, rows)
+
+
+def test_varlen_multi_pass():
+    """A workspace for one 2048-row window: the attention runs window by window across sequences."""
+    cfg = _cfg("passes", (1500, 3000, 200, 2300), 8, 2, 64, 64, 6)
+    _check(cfg, np.arange(cfg.T), max_rows_per_pass=2048)
+
+
+def test_varlen_single_sequence_equals_dense_path():
+    """B = 1: identical selections and outputs to msa_index_topk + msa_build_kv2q + msa_sparse_prefill."""
+    cfg = _cfg("single", (3333,), 16, 2, 128, 64, 5)
+    inp = synth.varlen_inputs(cfg)
+    t = {n: dev(inp[n]) for n in ("q", "k", "v", "q_idx", "k_idx")}
+    out_v, lse_v, bi_v = msa.msa_sparse_prefill_varlen(t["q"], t["k"], t["v"], t["q_idx"], t["k_idx"],
+                                                       inp["cu_seqlens"], 128, cfg.k)
+    bi = msa.msa_index_topk(t["q_idx"], t["k_idx"], 128, cfg.k)
+    kv = msa.msa_build_kv2q(bi, 128)
+    out, lse = msa.msa_sparse_prefill(t["q"], t["k"], t["v"], bi, kv)
+    torch.cuda.synchronize()
+    assert torch.equal(bi_v, bi)
+    assert torch.equal(out_v, out)
+    assert torch.equal(lse_v, lse)
