@@ -15,6 +15,7 @@ on a bounded sample of the same workload, and prints the same metric.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -42,6 +43,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["msa", "reference"], default="msa")
     ap.add_argument("--workload", default=synth.P128K.name, choices=sorted(synth.PREFILL_CONFIGS))
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch (varlen) prefill leg")
     ap.add_argument("--decode-workload", default=synth.DECODE64.name, choices=sorted(synth.DECODE_CONFIGS))
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-oracle sample time")
@@ -334,6 +336,42 @@ def gpu_arm(args, rank, world):
 
     pf_total, dec_total = replicas.max_over_ranks([sum(pf_ms), sum(dec_ms)], device=dev)
 
+    # packed-batch (varlen) prefill of the same model shape: 16 sequences, 131072 tokens in total
+    varlen = None
+    if not args.no_varlen:
+        vcfg = dataclasses.replace(synth.VARLEN128K, seed=replicas.replica_seed(synth.VARLEN128K.seed, rank))
+        vin = synth.varlen_inputs(vcfg)
+        vt = {n: to_dev(vin[n]) for n in ("q", "k", "v", "q_idx", "k_idx")}
+        v_out = torch.empty_like(vt["q"])
+        v_lse = torch.empty((vcfg.T, vcfg.H_q), dtype=torch.float32, device=dev)
+        v_bi = torch.empty((vcfg.H_kv, vcfg.T, vcfg.k), dtype=torch.int32, device=dev)
+        cu_p = vin["cu_seqlens"].ctypes.data_as(msa.api.ctypes.c_void_p)
+        v_ws = torch.empty(msa.api.lib.msa_sparse_prefill_varlen_workspace_size(
+            cu_p, len(vcfg.lens), vcfg.H_q, vcfg.H_kv, vcfg.d_h, vcfg.B_k, vcfg.k, 0), dtype=torch.uint8, device=dev)
+
+        def varlen_step():
+            msa.msa_sparse_prefill_varlen(vt["q"], vt["k"], vt["v"], vt["q_idx"], vt["k_idx"], vin["cu_seqlens"],
+                                          vcfg.B_k, vcfg.k, block_idx=v_bi, out=v_out, lse=v_lse, workspace=v_ws)
+
+        for _ in range(args.warmup):
+            varlen_step()
+        torch.cuda.synchronize()
+        if msa.msa_get_device_error(v_ws) != 0:
+            raise RuntimeError("device error in the varlen warm-up")
+        vev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for st in range(args.steps):
+            flush.zero_()
+            vev[st][0].record()
+            varlen_step()
+            vev[st][1].record()
+        torch.cuda.synchronize()
+        (vt_ms,) = replicas.max_over_ranks([sum(a.elapsed_time(b) for a, b in vev)], device=dev)
+        varlen = {"value": replicas.aggregate_rate(vcfg.T * args.steps, world, vt_ms / 1000.0), "unit": UNIT,
+                  "ms_per_step": vt_ms / args.steps, "workload": vcfg.name, "n_seq": len(vcfg.lens),
+                  "lens": f"{min(vcfg.lens)}..{max(vcfg.lens)} (seeded mix)",
+                  "note": "msa_sparse_prefill_varlen: index branch, inversion, attention and combine in one call"}
+        del vt, v_out, v_lse, v_bi, v_ws
+
     # end-to-end through the public API with host buffers (pinned), copies inside the timed region:
     # every step copies its inputs in and its output back; device inputs and outputs are double
     # buffered so step s+1's inputs stream in and step s-1's output streams out while step s computes
@@ -433,7 +471,7 @@ def gpu_arm(args, rank, world):
             "prefill_ms_per_step": pf_total / args.steps,
             "decode": ({"value": world * dcfg.B * args.steps / (dec_total / 1000.0), "unit": UNIT,
                         "ms_per_step": dec_total / args.steps} if dcfg else None),
-            "roofline": roof, "kernels": kstats, "cpu_baseline": cpu_base, "e2e": e2e,
+            "roofline": roof, "kernels": kstats, "cpu_baseline": cpu_base, "e2e": e2e, "varlen": varlen,
             "gpu_launches": int(launches), "clocks": clocks.summary(), "wall_s_timed": wall}
     print(json.dumps(line), flush=True)
 

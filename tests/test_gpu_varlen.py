@@ -84,3 +84,17 @@ def test_varlen_single_sequence_equals_dense_path():
     assert torch.equal(bi_v, bi)
     assert torch.equal(out_v, out)
     assert torch.equal(lse_v, lse)
+
+
+def test_varlen_full_size_sampled():
+    """The bench's packed batch (16 sequences, 131072 tokens, 64 q / 4 kv heads, d_h 128, k 16) on
+    sampled rows of every sequence."""
+    cfg = synth.VARLEN128K
+    cu = cfg.cu_seqlens()
+    rng = np.random.default_rng(11)
+    picks = []
+    for s in range(len(cfg.lens)):
+        n = cfg.lens[s]
+        local = np.unique(np.concatenate([[0, 127, 128, n - 1], rng.choice(n, 24, replace=False)]))
+        picks.append(int(cu[s]) + local[local < n])
+    _check(cfg, np.concatenate(picks))
