@@ -66,10 +66,10 @@ def load_peaks():
 # full launch is the per-row figure times its rows. A figure only applies to the sources it was
 # measured on: after any change to them the bench reports traffic as null.
 PROFILED_TRAFFIC = {
-    "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "b1c4a120f8dc8710",
-             "bytes_per_row": 307955.2, "capture": "profiles/sparse_attn_prefill_N32768.md (8192-row pass)"},
-    "combine": {"files": ("combine.cu", "common.cuh", "sm100.cuh"), "sha256_16": "930906627b9c1775",
-                "bytes_per_row": 282412.2, "capture": "profiles/combine_prefill_N32768.md (8192-row pass)"},
+    "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "b2d0b465db884013",
+             "bytes_per_row": 307763.5, "capture": "profiles/sparse_attn_prefill_N32768.md (8192-row pass)"},
+    "combine": {"files": ("combine.cu", "common.cuh", "sm100.cuh"), "sha256_16": "f4406ab7436d1d69",
+                "bytes_per_row": 282413.6, "capture": "profiles/combine_prefill_N32768.md (8192-row pass)"},
 }
 
 
