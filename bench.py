@@ -347,7 +347,8 @@ def gpu_arm(args, rank, world):
         v_bi = torch.empty((vcfg.H_kv, vcfg.T, vcfg.k), dtype=torch.int32, device=dev)
         cu_p = vin["cu_seqlens"].ctypes.data_as(msa.api.ctypes.c_void_p)
         v_ws = torch.empty(msa.api.lib.msa_sparse_prefill_varlen_workspace_size(
-            cu_p, len(vcfg.lens), vcfg.H_q, vcfg.H_kv, vcfg.d_h, vcfg.B_k, vcfg.k, 0), dtype=torch.uint8, device=dev)
+            cu_p, None, len(vcfg.lens), vcfg.H_q, vcfg.H_kv, vcfg.d_h, vcfg.B_k, vcfg.k, 0), dtype=torch.uint8,
+            device=dev)
 
         def varlen_step():
             msa.msa_sparse_prefill_varlen(vt["q"], vt["k"], vt["v"], vt["q_idx"], vt["k_idx"], vin["cu_seqlens"],

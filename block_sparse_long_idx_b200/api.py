@@ -55,8 +55,8 @@ SIGNATURES = [
     ("msa_sparse_decode_workspace_size", _sz, [_int, _i64, _int, _int, _int, _int, _int, _int]),
     ("msa_sparse_decode", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _int, _int, _int, _vp,
                                  _vp, _vp, _vp, _sz, _vp]),
-    ("msa_sparse_prefill_varlen_workspace_size", _sz, [_vp, _int, _int, _int, _int, _int, _int, _i64]),
-    ("msa_sparse_prefill_varlen", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int,
+    ("msa_sparse_prefill_varlen_workspace_size", _sz, [_vp, _vp, _int, _int, _int, _int, _int, _int, _i64]),
+    ("msa_sparse_prefill_varlen", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int,
                                          _vp, _vp, _vp, _vp, _sz, _vp]),
     ("msa_selftest_workspace_size", _sz, []),
     ("msa_selftest_wait_timeout", _int, [_vp, _sz, _i64, _vp]),
@@ -167,8 +167,9 @@ def msa_get_device_error(workspace: torch.Tensor, stream=None) -> int:
 
 def msa_sparse_prefill_varlen(q, k_, v, q_idx, k_idx, cu_seqlens, B_k: int = 128, k: int = 16, block_idx=None,
                               out=None, lse=None, want_lse: bool = True, workspace=None, max_rows_per_pass: int = 0,
-                              stream=None):
-    """Packed batch of independent sequences (cu_seqlens [B+1], host ints): index branch, inversion,
+                              stream=None, cu_seqlens_k=None):
+    """Packed batch of independent sequences (cu_seqlens [B+1], host ints, over the query rows;
+    cu_seqlens_k over the key rows when keys hold cached prefixes): index branch, inversion,
     attention and combine in one call. Returns (out [T, H_q, d_h], lse [T, H_q], block_idx [H_kv, T, k])."""
     for t, n in ((q, "q"), (k_, "k"), (v, "v"), (q_idx, "q_idx"), (k_idx, "k_idx")):
         _bf16(t, n)
@@ -177,18 +178,21 @@ def msa_sparse_prefill_varlen(q, k_, v, q_idx, k_idx, cu_seqlens, B_k: int = 128
     cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
     B = len(cu) - 1
     cu_p = cu.ctypes.data_as(ctypes.c_void_p)
+    cuk = None if cu_seqlens_k is None else np.ascontiguousarray(np.asarray(cu_seqlens_k, dtype=np.int32))
+    cuk_p = None if cuk is None else cuk.ctypes.data_as(ctypes.c_void_p)
     if block_idx is None:
         block_idx = torch.empty((H_kv, T, k), dtype=torch.int32, device=q.device)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((T, H_q), dtype=torch.float32, device=q.device)
-    need = lib.msa_sparse_prefill_varlen_workspace_size(cu_p, B, H_q, H_kv, d_h, B_k, k, max_rows_per_pass)
+    need = lib.msa_sparse_prefill_varlen_workspace_size(cu_p, cuk_p, B, H_q, H_kv, d_h, B_k, k, max_rows_per_pass)
     if need == 0:
         raise MsaError("msa_sparse_prefill_varlen_workspace_size", 1, "arguments rejected")
     ws = _workspace(need, q.device, workspace)
     _check("msa_sparse_prefill_varlen", lib.msa_sparse_prefill_varlen(
-        q.data_ptr(), k_.data_ptr(), v.data_ptr(), q_idx.data_ptr(), k_idx.data_ptr(), cu_p, B, H_q, H_kv, d_h, d_idx,
+        q.data_ptr(), k_.data_ptr(), v.data_ptr(), q_idx.data_ptr(), k_idx.data_ptr(), cu_p, cuk_p, B, H_q, H_kv, d_h,
+        d_idx,
         B_k, k, block_idx.data_ptr(), out.data_ptr(), _ptr(lse), ws.data_ptr(), ws.numel(), _stream(stream)))
     return out, lse, block_idx
 

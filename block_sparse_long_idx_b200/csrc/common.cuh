@@ -50,7 +50,8 @@ struct IndexTopkArgs {
     // packed batch of sequences (nullptr: one sequence of N rows): items are (sequence, tile pair)
     const int2* vitems = nullptr; // [n_vitems] (sequence, pair u), decreasing work first
     int n_vitems = 0;
-    const int32_t* cu = nullptr; // [B+1] first row of each sequence
+    const int32_t* cu = nullptr;   // [B+1] first query row of each sequence
+    const int32_t* cu_k = nullptr; // [B+1] first key row of each sequence (nullptr: same as cu)
 };
 cudaError_t launch_index_topk(const IndexTopkArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                               cudaStream_t s);
@@ -85,7 +86,9 @@ struct AttnArgs {
     int64_t row0;               // first row of the pass (= w0 * window)
     int64_t rows_pass;          // rows the partial buffers hold
     int* item_counter;          // work items claimed so far in this launch (zero at launch)
-    const int32_t* blk_tok = nullptr; // packed batch: first row of each global block (nullptr: b * B_k)
+    const int32_t* blk_tok = nullptr;  // packed batch: first key row of each global block (nullptr: b * B_k)
+    const int32_t* blk_qtok = nullptr; // packed batch: query-row coordinate of each block's first token
+                                       // (differs from blk_tok when keys and queries are packed apart)
     long long* timeline;        // optional: CTA 0 records clock64 per tile event (nullptr = off)
     int timeline_tiles;         // capacity in tiles (16 event slots per tile)
     uint16_t* o_part;           // [rows][k][H_q][d_h]
@@ -111,10 +114,12 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
-// Packed batch tables from cu[B+1] and blk_base[B+1] (global block of each sequence's block 0):
-// row_start[i], row_gb0[i] for every row, blk_tok[gb] for every global block.
-cudaError_t launch_varlen_tables(const int32_t* cu, const int32_t* blk_base, int B, int64_t T, int32_t nb_total,
-                                 int32_t* row_start, int32_t* row_gb0, int32_t* blk_tok, cudaStream_t s);
+// Packed batch tables from cu[B+1] (query rows), cu_k[B+1] (key rows) and blk_base[B+1] (global
+// block of each sequence's block 0): row_start[i], row_gb0[i] for every query row, blk_tok[gb] and
+// blk_qtok[gb] for every global block.
+cudaError_t launch_varlen_tables(const int32_t* cu, const int32_t* cu_k, const int32_t* blk_base, int B, int64_t T,
+                                 int32_t nb_total, int32_t* row_start, int32_t* row_gb0, int32_t* blk_tok,
+                                 int32_t* blk_qtok, cudaStream_t s);
 
 struct DecodeArgs {
     const uint16_t* q;

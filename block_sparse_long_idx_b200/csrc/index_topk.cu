@@ -42,31 +42,39 @@ struct IdxShared {
     int abort_flag;
 };
 
-// Work item j: group r = j % H_kv and a pair u of query tiles (2u, 2u+1) of one sequence, whose
-// rows are [row0, row0 + nrows) of the packed tensors (one sequence of N rows unless a.vitems).
+// Work item j: group r = j % H_kv and a pair u of query tiles of one sequence. The sequence's query
+// rows are [row0, row0 + nrows) of the query tensors and start at block t0 of the sequence (t0 > 0
+// when a prefix of the sequence is only in the key cache); its keys start at row krow0 of the key
+// tensors. Tile A is the sequence's block tA = t0 + 2u (rows row0 + 256u ..), tile B is tA + 1; a
+// row of tile t sees the blocks 0 .. t-1 in full. One sequence of N rows unless a.vitems.
 struct IdxItem {
-    int r, u, steps;
+    int r, u, steps, tA;
     bool tbv;
-    int row0, nrows;
+    int row0, nrows, krow0;
 };
 
 __device__ __forceinline__ IdxItem item_at(const IndexTopkArgs& a, int j, int n_pairs)
 {
     IdxItem it;
     it.r = j % a.H_kv;
+    int t0 = 0;
     if (a.vitems) {
         const int2 v = a.vitems[j / a.H_kv];
         it.u = v.y;
         it.row0 = a.cu[v.x];
         it.nrows = a.cu[v.x + 1] - it.row0;
+        it.krow0 = a.cu_k ? a.cu_k[v.x] : it.row0;
+        if (a.cu_k) t0 = (a.cu_k[v.x + 1] - it.krow0 - it.nrows) / kBk; // cached prefix, whole blocks
     } else {
         it.u = n_pairs - 1 - j / a.H_kv;
         it.row0 = 0;
         it.nrows = (int)a.N;
+        it.krow0 = 0;
     }
     const int n_qt = (it.nrows + kBk - 1) / kBk;
     it.tbv = (2 * it.u + 1) < n_qt;
-    it.steps = it.tbv ? 2 * it.u + 1 : 2 * it.u;
+    it.tA = t0 + 2 * it.u;
+    it.steps = it.tbv ? it.tA + 1 : it.tA;
     return it;
 }
 
@@ -147,7 +155,7 @@ __global__ void __launch_bounds__(384, 1)
                     mbar_arrive_expect_tx(&sh.kv_full[s], C::TILE_BYTES);
                     for (int c = 0; c < C::NKC; ++c)
                         tma_load_3d(sk + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &kmap, &sh.kv_full[s],
-                                    c * C::CHUNK_COLS, r, itm.row0 + b * kBk);
+                                    c * C::CHUNK_COLS, r, itm.krow0 + b * kBk);
                 }
                 ++item_cnt;
             }
@@ -186,7 +194,7 @@ __global__ void __launch_bounds__(384, 1)
                         const int col = ks * 16;
                         const uint32_t off = (col / C::CHUNK_COLS) * C::CHUNK_BYTES + (col % C::CHUNK_COLS) * 2;
                         const uint64_t kd = desc_kmajor(kb + off, C::SWB);
-                        if (b < 2 * u) mma_ss(tmem + buf * 128, desc_kmajor(aA + off, C::SWB), kd, idesc, ks > 0);
+                        if (b < itm.tA) mma_ss(tmem + buf * 128, desc_kmajor(aA + off, C::SWB), kd, idesc, ks > 0);
                         if (tbv) mma_ss(tmem + 256 + buf * 128, desc_kmajor(aB + off, C::SWB), kd, idesc, ks > 0);
                     }
                     tc_commit(&sh.kv_empty[s]);
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(384, 1)
             const IdxItem itm = item_at(a, j, n_pairs);
             const int r = itm.r, u = itm.u, steps = itm.steps;
             const bool tbv = itm.tbv;
-            const int tile = 2 * u + e;
+            const int tile = itm.tA + e; // the sequence's block of this tile's rows
             const bool active = (e == 0) || tbv;
             TopkList list;
             list.init(a.k - 1);
@@ -222,7 +230,7 @@ __global__ void __launch_bounds__(384, 1)
                     break;
                 }
                 tc_fence_after();
-                if (active && (e == 1 || b < 2 * u)) {
+                if (active && (e == 1 || b < itm.tA)) {
                     const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (e ? 256 : 0) + buf * 128;
                     float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, m2 = -CUDART_INF_F, m3 = -CUDART_INF_F;
 #pragma unroll
@@ -247,7 +255,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (!ok) break;
             if (active) {
-                const int il = tile * kBk + row; // row within its sequence
+                const int il = (2 * u + e) * kBk + row; // row among the sequence's query rows
                 if (il < itm.nrows)
                     emit_selection(list, tile, a.k, a.block_idx + ((int64_t)r * a.N + itm.row0 + il) * a.k);
             }

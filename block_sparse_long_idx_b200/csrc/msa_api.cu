@@ -312,7 +312,7 @@ static msa_status run_passes(const uint8_t* kvb, const msa_kv2q_layout* L, int64
                              const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
                              int64_t wins_per_pass, int64_t rows_pass, uint16_t* o_part, float* lse_part,
                              msa_bf16* out, float* lse, void* workspace, cudaStream_t s, const int32_t* blk_tok,
-                             const int32_t* row_start)
+                             const int32_t* row_start, const int32_t* blk_qtok = nullptr)
 {
     for (int64_t w0 = 0; w0 < L->n_windows; w0 += wins_per_pass) {
         const int64_t w1 = w0 + wins_per_pass < L->n_windows ? w0 + wins_per_pass : L->n_windows;
@@ -331,6 +331,7 @@ static msa_status run_passes(const uint8_t* kvb, const msa_kv2q_layout* L, int64
         a.rows_pass = rows_pass;
         a.item_counter = (int*)workspace + 4; // inside the error-word region, reset for every pass
         a.blk_tok = blk_tok;
+        a.blk_qtok = blk_qtok;
         a.timeline = nullptr;
         a.timeline_tiles = 0;
         a.o_part = o_part;
@@ -445,56 +446,66 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
 
 namespace {
 
-// Host-side plan of a packed batch: global block bases and the index work items (sequence, tile
-// pair) in decreasing work order.
+// Host-side plan of a packed batch: global block bases (key blocks of every sequence) and the index
+// work items (sequence, query tile pair) in decreasing work order.
 struct VarlenPlan {
     int B = 0;
-    int64_t T = 0, NB = 0;
-    std::vector<int32_t> head; // [cu (B+1) | blk_base (B+1) | vitems (2 * n_vitems)], copied to the device
+    int64_t T = 0, Tk = 0, NB = 0;
+    std::vector<int32_t> head; // [cu (B+1) | cu_k (B+1) | blk_base (B+1) | vitems (2 * n_vitems)]
     int n_vitems = 0;
-    size_t off_cu = 0, off_base = 0, off_items = 0, head_bytes = 0;
+    size_t off_cu = 0, off_cuk = 0, off_base = 0, off_items = 0, head_bytes = 0;
 };
 
-msa_status varlen_plan(const int32_t* cu, int B, VarlenPlan& p)
+msa_status varlen_plan(const int32_t* cu, const int32_t* cu_k, int B, VarlenPlan& p)
 {
-    if (!cu || B < 1 || cu[0] != 0) return MSA_ERR_INVALID_ARG;
-    for (int s = 0; s < B; ++s)
-        if (cu[s + 1] < cu[s]) return MSA_ERR_INVALID_ARG;
+    if (!cu || B < 1 || cu[0] != 0 || (cu_k && cu_k[0] != 0)) return MSA_ERR_INVALID_ARG;
+    if (!cu_k) cu_k = cu;
+    for (int s = 0; s < B; ++s) {
+        const int32_t nq = cu[s + 1] - cu[s], nk = cu_k[s + 1] - cu_k[s];
+        if (nq < 0 || nk < nq) return MSA_ERR_INVALID_ARG;       // keys cover the queries' positions
+        if ((nk - nq) % kBk != 0) return MSA_ERR_UNSUPPORTED;   // cached prefix in whole blocks
+    }
     p.B = B;
     p.T = cu[B];
+    p.Tk = cu_k[B];
     if (p.T < 1) return MSA_ERR_INVALID_ARG;
-    if (p.T > kMaxN) return MSA_ERR_UNSUPPORTED;
+    if (p.T > kMaxN || p.Tk > kMaxN) return MSA_ERR_UNSUPPORTED;
     std::vector<int32_t> base(B + 1, 0);
-    std::vector<std::pair<int, int>> items; // (u, s)
+    std::vector<std::pair<int, std::pair<int, int>>> items; // (work, (s, u))
     for (int s = 0; s < B; ++s) {
-        const int n_qt = (cu[s + 1] - cu[s] + kBk - 1) / kBk;
-        base[s + 1] = base[s] + n_qt;
-        for (int u = 0; u < (n_qt + 1) / 2; ++u) items.emplace_back(u, s);
+        const int nq = cu[s + 1] - cu[s], nk = cu_k[s + 1] - cu_k[s];
+        base[s + 1] = base[s] + (nk + kBk - 1) / kBk;
+        const int t0 = (nk - nq) / kBk, n_qt = (nq + kBk - 1) / kBk;
+        for (int u = 0; u < (n_qt + 1) / 2; ++u) items.push_back({t0 + 2 * u, {s, u}});
     }
     p.NB = base[B];
-    std::stable_sort(items.begin(), items.end(), [](const std::pair<int, int>& x, const std::pair<int, int>& y) {
-        return x.first > y.first; // most work first
-    });
+    std::stable_sort(items.begin(), items.end(),
+                     [](const std::pair<int, std::pair<int, int>>& x, const std::pair<int, std::pair<int, int>>& y) {
+                         return x.first > y.first; // most work first
+                     });
     p.n_vitems = (int)items.size();
+    const size_t cu_bytes = align_up((size_t)(B + 1) * 4, 16);
     p.off_cu = 0;
-    p.off_base = align_up((size_t)(B + 1) * 4, 16);
-    p.off_items = p.off_base + align_up((size_t)(B + 1) * 4, 16);
+    p.off_cuk = cu_bytes;
+    p.off_base = 2 * cu_bytes;
+    p.off_items = 3 * cu_bytes;
     p.head_bytes = align_up(p.off_items + (size_t)p.n_vitems * 8, 256);
     p.head.assign(p.head_bytes / 4, 0);
     for (int s = 0; s <= B; ++s) {
         p.head[p.off_cu / 4 + s] = cu[s];
+        p.head[p.off_cuk / 4 + s] = cu_k[s];
         p.head[p.off_base / 4 + s] = base[s];
     }
     for (int j = 0; j < p.n_vitems; ++j) {
-        p.head[p.off_items / 4 + 2 * j] = items[j].second;
-        p.head[p.off_items / 4 + 2 * j + 1] = items[j].first;
+        p.head[p.off_items / 4 + 2 * j] = items[j].second.first;
+        p.head[p.off_items / 4 + 2 * j + 1] = items[j].second.second;
     }
     return MSA_OK;
 }
 
 // Workspace carve-up of msa_sparse_prefill_varlen; rows_pass = 0 in the plan means "size query".
 struct VarlenWs {
-    size_t head, row_start, row_gb0, blk_tok, kv2q, kvtmp, parts, total;
+    size_t head, row_start, row_gb0, blk_tok, blk_qtok, kv2q, kvtmp, parts, total;
     int64_t rows_pass;
     msa_kv2q_layout L;
 };
@@ -511,6 +522,8 @@ msa_status varlen_ws(const VarlenPlan& p, int H_q, int H_kv, int d_h, int k, int
     w.row_gb0 = off;
     off += align_up((size_t)p.T * 4, 256);
     w.blk_tok = off;
+    off += align_up((size_t)p.NB * 4, 256);
+    w.blk_qtok = off;
     off += align_up((size_t)p.NB * 4, 256);
     w.kv2q = off;
     off += align_up(w.L.total_bytes, 256);
@@ -537,19 +550,20 @@ msa_status varlen_ws(const VarlenPlan& p, int H_q, int H_kv, int d_h, int k, int
 
 extern "C" {
 
-size_t msa_sparse_prefill_varlen_workspace_size(const int32_t* cu_seqlens, int B, int H_q, int H_kv, int d_h, int B_k,
-                                                int k, int64_t max_rows_per_pass)
+size_t msa_sparse_prefill_varlen_workspace_size(const int32_t* cu_seqlens, const int32_t* cu_seqlens_k, int B, int H_q,
+                                                int H_kv, int d_h, int B_k, int k, int64_t max_rows_per_pass)
 {
     VarlenPlan p;
     VarlenWs w;
-    if (B_k != kBk || H_q < 1 || H_kv < 1 || d_h < 1 || varlen_plan(cu_seqlens, B, p) != MSA_OK ||
+    if (B_k != kBk || H_q < 1 || H_kv < 1 || d_h < 1 || varlen_plan(cu_seqlens, cu_seqlens_k, B, p) != MSA_OK ||
         varlen_ws(p, H_q, H_kv, d_h, k, max_rows_per_pass, 0, w) != MSA_OK)
         return 0;
     return w.total;
 }
 
 msa_status msa_sparse_prefill_varlen(const msa_bf16* q, const msa_bf16* kk, const msa_bf16* v, const msa_bf16* q_idx,
-                                     const msa_bf16* k_idx, const int32_t* cu_seqlens, int B, int H_q, int H_kv,
+                                     const msa_bf16* k_idx, const int32_t* cu_seqlens, const int32_t* cu_seqlens_k,
+                                     int B, int H_q, int H_kv,
                                      int d_h, int d_idx, int B_k, int k, int32_t* block_idx, msa_bf16* out, float* lse,
                                      void* workspace, size_t workspace_bytes, msa_stream_t stream)
 {
@@ -564,34 +578,37 @@ msa_status msa_sparse_prefill_varlen(const msa_bf16* q, const msa_bf16* kk, cons
         !(d_idx == 32 || d_idx == 64 || d_idx == 128) || H_kv > 65535)
         return MSA_ERR_UNSUPPORTED;
     VarlenPlan p;
-    if (msa_status st = varlen_plan(cu_seqlens, B, p)) return st;
+    if (msa_status st = varlen_plan(cu_seqlens, cu_seqlens_k, B, p)) return st;
     VarlenWs w;
     if (msa_status st = varlen_ws(p, H_q, H_kv, d_h, k, 0, workspace_bytes, w)) return st;
     if (injected("msa_sparse_prefill_varlen")) return MSA_ERR_CUDA;
-    const int64_t T = p.T;
+    const int64_t T = p.T, Tk = p.Tk;
     CUtensorMap qim, kim, qmap, kmap, vmap;
     const uint32_t box0 = d_idx < 64 ? (uint32_t)d_idx : 64u;
     const CUtensorMapSwizzle sw = d_idx == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     if (!make_map_3d(&qim, q_idx, d_idx, H_kv, T, box0, 1, kBk, sw) ||
-        !make_map_3d(&kim, k_idx, d_idx, H_kv, T, box0, 1, kBk, sw) ||
+        !make_map_3d(&kim, k_idx, d_idx, H_kv, Tk, box0, 1, kBk, sw) ||
         !make_map_3d(&qmap, q, d_h, H_q, T, 64, G, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_3d(&kmap, kk, d_h, H_kv, T, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_3d(&vmap, v, d_h, H_kv, T, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_map_3d(&kmap, kk, d_h, H_kv, Tk, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d(&vmap, v, d_h, H_kv, Tk, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B))
         return MSA_ERR_INVALID_ARG;
 
     cudaStream_t s = (cudaStream_t)stream;
     uint8_t* ws = (uint8_t*)workspace;
     const int32_t* d_cu = (const int32_t*)(ws + w.head + p.off_cu);
+    const int32_t* d_cuk = (const int32_t*)(ws + w.head + p.off_cuk);
     const int32_t* d_base = (const int32_t*)(ws + w.head + p.off_base);
     const int2* d_items = (const int2*)(ws + w.head + p.off_items);
     int32_t* row_start = (int32_t*)(ws + w.row_start);
     int32_t* row_gb0 = (int32_t*)(ws + w.row_gb0);
     int32_t* blk_tok = (int32_t*)(ws + w.blk_tok);
+    int32_t* blk_qtok = (int32_t*)(ws + w.blk_qtok);
     if (msa_status st = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st;
     if (msa_status st = cuda_status(cudaMemcpyAsync(ws + w.head, p.head.data(), p.head_bytes, cudaMemcpyHostToDevice, s),
                                     "copying the batch plan"))
         return st;
-    if (msa_status st = cuda_status(launch_varlen_tables(d_cu, d_base, B, T, (int32_t)p.NB, row_start, row_gb0, blk_tok, s),
+    if (msa_status st = cuda_status(launch_varlen_tables(d_cu, d_cuk, d_base, B, T, (int32_t)p.NB, row_start, row_gb0,
+                                                         blk_tok, blk_qtok, s),
                                     "varlen tables launch"))
         return st;
     // index branch over (sequence, tile pair) items
@@ -599,6 +616,7 @@ msa_status msa_sparse_prefill_varlen(const msa_bf16* q, const msa_bf16* kk, cons
     ia.vitems = d_items;
     ia.n_vitems = p.n_vitems;
     ia.cu = d_cu;
+    ia.cu_k = d_cuk;
     trace_begin(s);
     const cudaError_t ei = launch_index_topk(ia, qim, kim, s);
     trace_end(s, MSA_KERNEL_INDEX_TOPK);
@@ -611,7 +629,7 @@ msa_status msa_sparse_prefill_varlen(const msa_bf16* q, const msa_bf16* kk, cons
     uint16_t* o_part = (uint16_t*)(ws + w.parts);
     float* lse_part = (float*)(ws + w.parts + align_up((size_t)w.rows_pass * k * H_q * d_h * 2, 256));
     return run_passes(ws + w.kv2q, &w.L, T, H_q, H_kv, d_h, k, qmap, kmap, vmap, wins_per_pass, w.rows_pass, o_part,
-                      lse_part, out, lse, workspace, s, blk_tok, row_start);
+                      lse_part, out, lse, workspace, s, blk_tok, row_start, blk_qtok);
 }
 
 // ------------------------------------------------------------------------------------ decode

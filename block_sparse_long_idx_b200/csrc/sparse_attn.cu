@@ -59,7 +59,7 @@ struct TileRec {
     int32_t r, b;  // GQA group, KV block
     int32_t npos;  // positions in the tile (1 .. 128/G); -1 marks the end of the CTA's work
     int32_t flags; // bit 0: first tile of its item, bit 1: last tile, bit 2: K/V stage of the item
-    int32_t tok0;  // first row of block b (b * 128, or from the block table of a packed batch)
+    int32_t tok0;  // query-row coordinate of block b's first token (b * 128 for one sequence)
 };
 
 struct AttnShared {
@@ -213,7 +213,8 @@ __global__ void __launch_bounds__(512, 1)
                 if (!ok) break;
                 const int32_t* ent = a.entries + (int64_t)item.r * Nk + item.start;
                 const int ntiles = (item.len + PPT - 1) / PPT;
-                const int tok0 = a.blk_tok ? a.blk_tok[item.b] : item.b * kBk;
+                // query-row coordinate of the block's first token (for the causal mask on the diagonal block)
+                const int tok0 = a.blk_qtok ? a.blk_qtok[item.b] : a.blk_tok ? a.blk_tok[item.b] : item.b * kBk;
                 for (int t = 0; t < ntiles; ++t, ++qt) {
                     const int qs = qt % NQ, rs = qt % kRing;
                     const int npos = min(PPT, item.len - t * PPT);

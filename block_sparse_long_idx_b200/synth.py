@@ -181,16 +181,28 @@ class VarlenConfig:
     B_k: int
     k: int
     seed: int
+    prefix: tuple = ()  # per sequence, tokens already in the key cache before its query rows (whole blocks)
 
     @property
     def T(self) -> int:
         return int(sum(self.lens))
 
+    def prefixes(self) -> np.ndarray:
+        return np.asarray(self.prefix if self.prefix else (0,) * len(self.lens), dtype=np.int64)
+
+    @property
+    def Tk(self) -> int:
+        return int(self.T + self.prefixes().sum())
+
     def cu_seqlens(self) -> np.ndarray:
         return np.concatenate([[0], np.cumsum(self.lens)]).astype(np.int32)
 
+    def cu_seqlens_k(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(np.asarray(self.lens) + self.prefixes())]).astype(np.int32)
+
     def packed(self) -> "PrefillConfig":
-        return PrefillConfig(self.name, N=self.T, H_q=self.H_q, H_kv=self.H_kv, d_h=self.d_h, d_idx=self.d_idx,
+        """The key-side tensors: all tokens (cached prefixes and query rows) of all sequences."""
+        return PrefillConfig(self.name, N=self.Tk, H_q=self.H_q, H_kv=self.H_kv, d_h=self.d_h, d_idx=self.d_idx,
                              B_k=self.B_k, k=self.k, seed=self.seed)
 
 
@@ -264,10 +276,18 @@ def prefill_inputs(cfg: PrefillConfig) -> dict:
 
 
 def varlen_inputs(cfg: VarlenConfig) -> dict:
-    """Packed tensors of all sequences ([T, heads, dim], as prefill_inputs of one T-token sequence)
-    plus cu_seqlens [B+1] int32; every sequence is an independent causal problem."""
+    """Packed tensors of all sequences plus cu_seqlens [B+1] (query rows) and cu_seqlens_k [B+1] (key
+    rows); every sequence is an independent causal problem. k, v, k_idx hold every token of every
+    sequence ([Tk, heads, dim]); q, q_idx hold each sequence's last len (query) tokens ([T, ...])."""
     d = prefill_inputs(cfg.packed())
-    d["cu_seqlens"] = cfg.cu_seqlens()
+    cu, cuk = cfg.cu_seqlens(), cfg.cu_seqlens_k()
+    pre = cfg.prefixes()
+    if pre.any():
+        take = np.concatenate([np.arange(cuk[s] + pre[s], cuk[s + 1]) for s in range(len(cfg.lens))]).astype(np.int64)
+        d["q"] = np.ascontiguousarray(d["q"][take])
+        d["q_idx"] = np.ascontiguousarray(d["q_idx"][take])
+    d["cu_seqlens"] = cu
+    d["cu_seqlens_k"] = cuk
     return d
 
 

@@ -207,32 +207,41 @@ MSA_API msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* k, cons
 /* ------------------------------------------------------------------------------------------
  * Packed-batch (varlen) prefill: the whole forward for B independent sequences  [EXPL 05, ABS]
  *
- * Sequence s holds rows cu_seqlens[s] .. cu_seqlens[s+1]-1 of the packed tensors. Each sequence is
- * its own causal problem with the definitions of msa_index_topk and msa_sparse_prefill applied to
- * its rows alone: its blocks are numbered from 0 at its first row, rows never see another
- * sequence's tokens. One call runs the index branch, the inversion (keyed on the blocks of all
- * sequences), the attention and the combine.
+ * Sequence s has query rows cu_seqlens[s] .. cu_seqlens[s+1]-1 of the packed query tensors and key
+ * rows cu_seqlens_k[s] .. cu_seqlens_k[s+1]-1 of the packed key tensors. Each sequence is its own
+ * causal problem with the definitions of msa_index_topk and msa_sparse_prefill applied to its
+ * tokens alone: its blocks are numbered from 0 at its first token, rows never see another
+ * sequence's tokens. When a sequence has more keys than queries (chunked prefill continuing from a
+ * KV cache: the keys hold the cached prefix followed by the chunk), its queries are its LAST
+ * positions: query row r of the sequence sits at position (len_k - len_q) + r, and the prefix
+ * length len_k - len_q must be a whole number of blocks. One call runs the index branch, the
+ * inversion (keyed on the blocks of all sequences), the attention and the combine.
  *
- *   q        : [T, H_q, d_h] bf16; k, v : [T, H_kv, d_h] bf16; q_idx, k_idx : [T, H_kv, d_idx] bf16
- *              (T = cu_seqlens[B], all 16-byte aligned)
- *   cu_seqlens: HOST array [B+1], cu_seqlens[0] = 0, non-decreasing (empty sequences allowed);
- *              read before the call returns (it sizes the schedule, which is copied to the device)
+ *   q, q_idx : [T, H_q, d_h], [T, H_kv, d_idx] bf16, T = cu_seqlens[B] query rows
+ *   k, v, k_idx : [Tk, H_kv, d_h], [Tk, H_kv, d_idx] bf16, Tk = cu_seqlens_k[B] key rows
+ *              (all 16-byte aligned)
+ *   cu_seqlens, cu_seqlens_k: HOST arrays [B+1] starting at 0, non-decreasing (empty sequences
+ *              allowed); cu_seqlens_k may be NULL (keys packed like the queries, no prefixes);
+ *              read before the call returns (they size the schedule, which is copied to the device)
  *   block_idx: [H_kv, T, k] int32 out: each row's selection as block indices local to its
  *              sequence, ascending, -1 padded (as msa_index_topk for that sequence alone)
  *   out      : [T, H_q, d_h] bf16 out;  lse : [T, H_q] fp32 out, or NULL
  *   workspace: >= msa_sparse_prefill_varlen_workspace_size(cu_seqlens, B, ..., max_rows_per_pass)
  *              bytes, 256-byte aligned, caller-owned; smaller workspaces run the attention in passes
  *              of whole query windows, down to one window
- * Errors: MSA_ERR_INVALID_ARG (NULL/misaligned pointers, bad cu_seqlens), MSA_ERR_UNSUPPORTED
- * (shapes outside this build), MSA_ERR_WORKSPACE, MSA_ERR_CUDA; device checks as msa_sparse_prefill.
+ * Errors: MSA_ERR_INVALID_ARG (NULL/misaligned pointers, bad cu_seqlens, fewer keys than queries
+ * in a sequence), MSA_ERR_UNSUPPORTED (shapes outside this build, a prefix that is not a whole
+ * number of blocks), MSA_ERR_WORKSPACE, MSA_ERR_CUDA; device checks as msa_sparse_prefill.
  * msa_sparse_prefill_varlen_workspace_size returns 0 for arguments the call would reject.
  * ------------------------------------------------------------------------------------------ */
-MSA_API size_t msa_sparse_prefill_varlen_workspace_size(const int32_t* cu_seqlens, int B, int H_q, int H_kv, int d_h,
-                                                        int B_k, int k, int64_t max_rows_per_pass);
+MSA_API size_t msa_sparse_prefill_varlen_workspace_size(const int32_t* cu_seqlens, const int32_t* cu_seqlens_k, int B,
+                                                        int H_q, int H_kv, int d_h, int B_k, int k,
+                                                        int64_t max_rows_per_pass);
 
 MSA_API msa_status msa_sparse_prefill_varlen(const msa_bf16* q, const msa_bf16* k, const msa_bf16* v,
                                              const msa_bf16* q_idx, const msa_bf16* k_idx, const int32_t* cu_seqlens,
-                                             int B, int H_q, int H_kv, int d_h, int d_idx, int B_k, int kk,
+                                             const int32_t* cu_seqlens_k, int B, int H_q, int H_kv, int d_h, int d_idx,
+                                             int B_k, int kk,
                                              int32_t* block_idx, msa_bf16* out, float* lse, void* workspace,
                                              size_t workspace_bytes, msa_stream_t stream);
 

@@ -124,12 +124,16 @@ class Oracle:
         out, lse = self.attend_rows(inputs["q"], inputs["k"], inputs["v"], rows, sel, B_k, n_threads)
         return sel, out, lse
 
-    def prefill_varlen_rows(self, inputs: dict, cu_seqlens, rows, B_k: int, k: int, n_threads: int = 0):
-        """Packed batch of independent sequences (cu_seqlens [B+1]): each sequence is its own causal
-        problem, so each row is answered by the single-sequence path on its sequence's slice of the
-        packed tensors, in the sequence's local indices. Returns (sel [n, H_kv, k] with local block
-        ids, out, lse) for the given global rows."""
+    def prefill_varlen_rows(self, inputs: dict, cu_seqlens, rows, B_k: int, k: int, n_threads: int = 0,
+                            cu_seqlens_k=None):
+        """Packed batch of independent sequences: query rows packed by cu_seqlens [B+1] (q, q_idx),
+        keys packed by cu_seqlens_k [B+1] (k, v, k_idx; default: like the queries). A sequence with
+        more keys than queries holds a cached prefix: its query rows are its last positions. Each
+        sequence is its own causal problem, so each row is answered by the single-sequence path on
+        that sequence's tokens (query rows placed at their positions), in the sequence's local block
+        indices. Returns (sel [n, H_kv, k], out, lse) for the given global query rows."""
         cu = np.asarray(cu_seqlens, dtype=np.int64)
+        cuk = cu if cu_seqlens_k is None else np.asarray(cu_seqlens_k, dtype=np.int64)
         rows = np.asarray(rows, dtype=np.int64)
         seq = np.searchsorted(cu, rows, side="right") - 1
         H_kv = inputs["k_idx"].shape[1]
@@ -139,9 +143,15 @@ class Oracle:
         lse = np.empty((len(rows), H_q), dtype=np.float64)
         for s in np.unique(seq):
             lo, hi = int(cu[s]), int(cu[s + 1])
+            klo, khi = int(cuk[s]), int(cuk[s + 1])
+            prefix = (khi - klo) - (hi - lo)
+            part = {n: np.ascontiguousarray(inputs[n][klo:khi]) for n in ("k", "v", "k_idx")}
+            for n in ("q", "q_idx"):  # query rows at their positions; cached positions are never queried
+                full = np.zeros((khi - klo,) + inputs[n].shape[1:], dtype=inputs[n].dtype)
+                full[prefix:] = inputs[n][lo:hi]
+                part[n] = full
             pick = np.nonzero(seq == s)[0]
-            part = {n: np.ascontiguousarray(inputs[n][lo:hi]) for n in ("q", "k", "v", "q_idx", "k_idx")}
-            s_sel, s_out, s_lse = self.prefill_rows(part, rows[pick] - lo, B_k, k, n_threads)
+            s_sel, s_out, s_lse = self.prefill_rows(part, rows[pick] - lo + prefix, B_k, k, n_threads)
             sel[pick], out[pick], lse[pick] = s_sel, s_out, s_lse
         return sel, out, lse
 

@@ -270,6 +270,32 @@ def check_varlen_matches_dense_per_sequence(o):
         assert np.max(np.abs(lse[lo:hi] - want_lse)) < 1e-12, s
 
 
+def check_varlen_cached_prefix_matches_dense(o):
+    """Queries that continue a cached prefix: each sequence's chunk rows equal the dense brute force of
+    the whole sequence at those positions (prefix tokens are keys only, never queried)."""
+    lens_k = [48, 80, 130, 64]
+    prefix = [32, 0, 64, 48]  # whole blocks of B_k = 16
+    H_q, H_kv, d_h, d_idx, B_k, k = 4, 2, 8, 8, 16, 3
+    cuk = np.concatenate([[0], np.cumsum(lens_k)])
+    lens_q = [a - b for a, b in zip(lens_k, prefix)]
+    cu = np.concatenate([[0], np.cumsum(lens_q)])
+    full = _attn_inputs(int(cuk[-1]), H_q, H_kv, d_h, d_idx, 21)
+    take = np.concatenate([np.arange(cuk[s] + prefix[s], cuk[s + 1]) for s in range(len(lens_k))])
+    inp = {"k": full["k"], "v": full["v"], "k_idx": full["k_idx"], "q": full["q"][take], "q_idx": full["q_idx"][take]}
+    sel, out, lse = o.prefill_varlen_rows(inp, cu, np.arange(int(cu[-1])), B_k, k, cu_seqlens_k=cuk)
+    for s in range(len(lens_k)):
+        klo, khi = int(cuk[s]), int(cuk[s + 1])
+        n = khi - klo
+        part = {name: full[name][klo:khi] for name in full}
+        want_sel = ref.dense_selection(part["q_idx"], part["k_idx"], B_k, k)[:, prefix[s]:]
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        assert np.array_equal(np.ascontiguousarray(sel[lo:hi].transpose(1, 0, 2)), want_sel), s
+        all_sel = ref.dense_selection(part["q_idx"], part["k_idx"], B_k, k)
+        want, want_lse = ref.masked_attention(part["q"], part["k"], part["v"], ref.selection_mask(all_sel, n, B_k))
+        assert np.max(np.abs(out[lo:hi] - want[prefix[s]:])) < 1e-12, s
+        assert np.max(np.abs(lse[lo:hi] - want_lse[prefix[s]:])) < 1e-12, s
+
+
 ALL_CHECKS = [
     check_selection_bruteforce,
     check_selection_ties_closed_form,
@@ -284,4 +310,5 @@ ALL_CHECKS = [
     check_kv2q_bruteforce,
     check_decode_matches_prefill_row,
     check_varlen_matches_dense_per_sequence,
+    check_varlen_cached_prefix_matches_dense,
 ]

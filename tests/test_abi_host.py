@@ -130,18 +130,27 @@ def test_varlen_validation_and_sizes(msa):
         return a, a.ctypes.data_as(c_vp)
 
     good, gp = cu(0, 100, 100, 1000, 4096)
-    sz = lib.msa_sparse_prefill_varlen_workspace_size(gp, 4, 16, 2, 128, 128, 8, 0)
+    sz = lib.msa_sparse_prefill_varlen_workspace_size(gp, None, 4, 16, 2, 128, 128, 8, 0)
     assert sz > 0
     # fewer rows per pass -> smaller workspace, never below one window
-    assert 0 < lib.msa_sparse_prefill_varlen_workspace_size(gp, 4, 16, 2, 128, 128, 8, 2048) <= sz
+    assert 0 < lib.msa_sparse_prefill_varlen_workspace_size(gp, None, 4, 16, 2, 128, 128, 8, 2048) <= sz
     for bad in ((1, 100), (0, 50, 40), (0, 0)):
         b, bp = cu(*bad)
-        assert lib.msa_sparse_prefill_varlen_workspace_size(bp, len(bad) - 1, 16, 2, 128, 128, 8, 0) == 0
-        assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, bp, len(bad) - 1, 16, 2, 128, 64, 128, 8, P2, P, None, WS,
-                                             sz, None) == INVALID
-    args = (P, P, P, P, P, gp, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS)
+        assert lib.msa_sparse_prefill_varlen_workspace_size(bp, None, len(bad) - 1, 16, 2, 128, 128, 8, 0) == 0
+        assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, bp, None, len(bad) - 1, 16, 2, 128, 64, 128, 8, P2, P,
+                                             None, WS, sz, None) == INVALID
+    args = (P, P, P, P, P, gp, None, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS)
     assert lib.msa_sparse_prefill_varlen(*args, 256, None) == WORKSPACE
-    assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, gp, 4, 16, 2, 96, 64, 128, 8, P2, P, None, WS, sz,
+    assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, gp, None, 4, 16, 2, 96, 64, 128, 8, P2, P, None, WS, sz,
                                          None) == UNSUPPORTED
-    assert lib.msa_sparse_prefill_varlen(P + 8, P, P, P, P, gp, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS, sz,
+    assert lib.msa_sparse_prefill_varlen(P + 8, P, P, P, P, gp, None, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS, sz,
+                                         None) == INVALID
+    # keys with cached prefixes: whole blocks only, never fewer keys than queries
+    ok_k, okp = cu(0, 228, 356, 1256, 4352)      # prefixes 128, 128, 0, 0 ... per sequence differences
+    assert lib.msa_sparse_prefill_varlen_workspace_size(gp, okp, 4, 16, 2, 128, 128, 8, 0) > 0
+    part, pp = cu(0, 150, 150, 1050, 4146)       # prefix 50: not a whole block
+    assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, gp, pp, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS, sz,
+                                         None) == UNSUPPORTED
+    short, sp = cu(0, 50, 50, 950, 4042)         # fewer keys than queries
+    assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, gp, sp, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS, sz,
                                          None) == INVALID
