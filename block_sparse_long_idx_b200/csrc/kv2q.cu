@@ -175,45 +175,75 @@ __global__ void kv2q_relative_kernel(Kv2qArgs a, const int32_t* group_starts)
 }
 
 // ------------------------------------------------------------------------------------ 3. scatter
-__global__ void kv2q_scatter_kernel(Kv2qArgs a)
+// The window's rows are split into nsub consecutive sub-ranges, one warp each. A warp first counts
+// its sub-range's entries per block; the starting position of warp s in block b's list is the
+// window's base for b plus the counts of warps 0 .. s-1, so the warps then scatter concurrently and
+// every list stays row-sorted.
+__device__ __forceinline__ int32_t scatter_block(const Kv2qArgs& a, int32_t b, int64_t i)
 {
-    extern __shared__ int32_t next_pos[]; // [nb] next write position of each block's list in this window
+    if (b < 0) return -1;
+    const int64_t il = a.row_start ? i - a.row_start[i] : i;
+    const int32_t g0 = a.row_gb0 ? a.row_gb0[i] : 0;
+    return (b + g0 >= a.nb || (int64_t)b * kBk > il) ? -1 : b + g0; // invalid ones: reported by the count pass
+}
+
+__global__ void kv2q_scatter_kernel(Kv2qArgs a, int nsub)
+{
+    extern __shared__ int32_t next_pos[]; // [nsub][nb] next write position of each warp in each block's list
     const int w = blockIdx.x, r = blockIdx.y;
-    const int lane = threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t* bases = a.bases + (int64_t)r * a.nb * a.n_windows;
-    for (int b = lane; b < a.nb; b += 32) next_pos[b] = bases[(int64_t)b * a.n_windows + w];
-    __syncwarp();
     const int64_t row_lo = (int64_t)w * a.window;
     const int64_t row_hi = min(a.N, row_lo + a.window);
+    const int64_t sub_rows = (row_hi - row_lo + nsub - 1) / nsub;
+    const int64_t my_lo = min(row_hi, row_lo + warp * sub_rows), my_hi = min(row_hi, my_lo + sub_rows);
     const int32_t* sel = a.block_idx + (int64_t)r * a.N * a.k;
     int32_t* ent = a.entries + (int64_t)r * a.N * a.k;
     const int rows_per_step = 32 / a.k;
     const unsigned lt_mask = (1u << lane) - 1u;
     const int slot = lane % a.k;
     const bool lane_used = lane < rows_per_step * a.k;
+    int32_t* mine = next_pos + (int64_t)warp * a.nb;
+    for (int b = threadIdx.x; b < nsub * a.nb; b += blockDim.x) next_pos[b] = 0;
+    __syncthreads();
+    // 1. count this warp's entries per block
+    for (int64_t i0 = my_lo; i0 < my_hi; i0 += rows_per_step) {
+        const int64_t i = i0 + lane / a.k;
+        const int32_t b = scatter_block(a, lane_used && i < my_hi ? sel[i * a.k + slot] : -1, i);
+        const unsigned peers = __match_any_sync(0xffffffffu, b);
+        if (b >= 0 && (peers & lt_mask) == 0) mine[b] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // 2. starting positions: window base + counts of the earlier sub-ranges
+    for (int b = threadIdx.x; b < a.nb; b += blockDim.x) {
+        int32_t pos = bases[(int64_t)b * a.n_windows + w];
+        for (int s2 = 0; s2 < nsub; ++s2) {
+            const int32_t c = next_pos[(int64_t)s2 * a.nb + b];
+            next_pos[(int64_t)s2 * a.nb + b] = pos;
+            pos += c;
+        }
+    }
+    __syncthreads();
+    // 3. scatter, rows in ascending order within the sub-range
     constexpr int kAhead = 8; // selection loads in flight per lane
-    for (int64_t i00 = row_lo; i00 < row_hi; i00 += (int64_t)rows_per_step * kAhead) {
+    for (int64_t i00 = my_lo; i00 < my_hi; i00 += (int64_t)rows_per_step * kAhead) {
         int32_t bs[kAhead];
 #pragma unroll
         for (int u = 0; u < kAhead; ++u) {
             const int64_t i = i00 + (int64_t)u * rows_per_step + lane / a.k;
-            bs[u] = lane_used && i < row_hi ? sel[i * a.k + slot] : -1;
+            bs[u] = lane_used && i < my_hi ? sel[i * a.k + slot] : -1;
         }
 #pragma unroll
         for (int u = 0; u < kAhead; ++u) {
             const int64_t i = i00 + (int64_t)u * rows_per_step + lane / a.k;
-            int32_t b = bs[u];
-            if (b >= 0) {
-                const int64_t il = a.row_start ? i - a.row_start[i] : i;
-                const int32_t g0 = a.row_gb0 ? a.row_gb0[i] : 0;
-                b = (b + g0 >= a.nb || (int64_t)b * kBk > il) ? -1 : b + g0; // invalid ones: reported by the count pass
-            }
+            const int32_t b = scatter_block(a, bs[u], i);
             const unsigned peers = __match_any_sync(0xffffffffu, b);
             if (b >= 0) {
                 const unsigned before = peers & lt_mask;
-                ent[next_pos[b] + __popc(before)] = (int32_t)(i * a.k + slot);
+                ent[mine[b] + __popc(before)] = (int32_t)(i * a.k + slot);
                 __syncwarp(peers);
-                if (before == 0) next_pos[b] += __popc(peers);
+                if (before == 0) mine[b] += __popc(peers);
             }
             __syncwarp();
         }
@@ -261,7 +291,11 @@ cudaError_t launch_kv2q(const Kv2qArgs& a, cudaStream_t s)
     const size_t hist_bytes = (size_t)a.nb * sizeof(int32_t);
     cudaError_t e = cudaFuncSetAttribute(kv2q_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_bytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kv2q_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_bytes);
+    // scatter: up to 8 warps per (window, group), as many as their per-block positions fit in shared memory
+    int nsub = (int)((200 * 1024) / hist_bytes);
+    nsub = nsub < 1 ? 1 : nsub > 8 ? 8 : nsub;
+    const size_t scatter_bytes = (size_t)nsub * hist_bytes;
+    e = cudaFuncSetAttribute(kv2q_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scatter_bytes);
     if (e != cudaSuccess) return e;
 
     const int64_t n = (int64_t)a.H_kv * a.nb * a.n_windows;
@@ -279,7 +313,7 @@ cudaError_t launch_kv2q(const Kv2qArgs& a, cudaStream_t s)
     const int64_t nb256 = (n + 255) / 256;
     const int nsm_blocks = (int)(nb256 < 4096 ? nb256 : 4096);
     kv2q_relative_kernel<<<nsm_blocks, 256, 0, s>>>(a, group_starts);
-    kv2q_scatter_kernel<<<grid_wr, 32, hist_bytes, s>>>(a);
+    kv2q_scatter_kernel<<<grid_wr, 32 * nsub, scatter_bytes, s>>>(a, nsub);
     exclusive_scan(ItemsInWRB{a.counts, a.H_kv, a.nb, a.n_windows, a.chunk}, n, item_bases, partials, n_items_total,
                    s);
     kv2q_items_kernel<<<nsm_blocks, 256, 0, s>>>(a, item_bases, n_items_total);
