@@ -14,9 +14,12 @@
  * Conventions shared by every entry point
  *   - bf16 tensors are passed as uint16_t bit patterns (msa_bf16).
  *   - Every tensor pointer is a DEVICE pointer into memory the caller allocated and owns; the
- *     library never allocates, frees or retains memory and keeps no global state besides the
- *     cached driver entry point used to encode TMA descriptors.
- *   - All work is enqueued asynchronously on `stream`; nothing synchronises the host.
+ *     library never allocates, frees or retains memory. Its only global state: the cached driver
+ *     entry point used to encode TMA descriptors, the fixed scratch of msa_build_kv2q_static and
+ *     the tracing hooks (msa_trace_set, msa_launch_count).
+ *   - All work is enqueued asynchronously on `stream`. Exceptions: msa_get_device_error waits for
+ *     the stream, and msa_sparse_prefill_varlen copies its host-side schedule from pageable
+ *     memory (the copy may block the host until it is staged).
  *   - Arguments are validated on the host before anything is enqueued; a rejected call enqueues
  *     nothing and returns MSA_ERR_INVALID_ARG (bad pointer / shape / alignment),
  *     MSA_ERR_UNSUPPORTED (a valid shape this build has no kernel for) or MSA_ERR_WORKSPACE
@@ -129,7 +132,7 @@ MSA_API msa_status msa_index_topk(const msa_bf16* q_idx, const msa_bf16* k_idx, 
  *                                      covers at most `chunk` consecutive entries of one list.
  *   window_items int32 [n_windows + 1] first item of each window; the last value is the count
  *   (plus internal per-(r, b, window) counts used while building)
- * window = 0 / chunk = 0 select the defaults (2048 rows per window, chunk = window).
+ * window = 0 / chunk = 0 select the defaults (2048 rows per window, items of at most 512 entries).
  * ------------------------------------------------------------------------------------------ */
 typedef struct {
     int32_t r;     /* GQA group */
