@@ -154,3 +154,23 @@ def test_varlen_validation_and_sizes(msa):
     short, sp = cu(0, 50, 50, 950, 4042)         # fewer keys than queries
     assert lib.msa_sparse_prefill_varlen(P, P, P, P, P, gp, sp, 4, 16, 2, 128, 64, 128, 8, P2, P, None, WS, sz,
                                          None) == INVALID
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without the built CUDA library the package refuses to load: there is no CPU or PyTorch path."""
+    pkg = os.path.join(ROOT, "block_sparse_long_idx_b200")
+    code = (
+        "import sys, os, shutil\n"
+        "sys.path.insert(0, %r)\n"
+        "shutil.copytree(%r, os.path.join(%r, 'block_sparse_long_idx_b200'),\n"
+        "                ignore=shutil.ignore_patterns('*.so', '_build', '__pycache__'))\n"
+        "import block_sparse_long_idx_b200 as m\n"
+        "try:\n"
+        "    m.msa_index_topk\n"
+        "except ImportError as e:\n"
+        "    print('IMPORT_ERROR', 'no CPU or PyTorch fallback' in str(e))\n"
+        "else:\n"
+        "    print('LOADED')\n" % (str(tmp_path), pkg, str(tmp_path)))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
+                         cwd=str(tmp_path))
+    assert "IMPORT_ERROR True" in out.stdout, out.stdout + out.stderr
