@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(384, 1)
                 const int j = item_for_round(round, cta, P);
                 if (j >= n_items) break;
                 const IdxItem itm = item_at(a, j, n_pairs);
-                const int u = itm.u, steps = itm.steps;
+                const int steps = itm.steps;
                 const bool tbv = itm.tbv;
                 if (!poll_or_abort(&sh.q_full, item_cnt & 1, abort_flag, a.err, 3, kWaitLimit)) break;
                 tc_fence_after();
