@@ -198,7 +198,10 @@ __global__ void __launch_bounds__(32) decode_topk_kernel(DecodeArgs a, int nb_ma
 template <int DH>
 struct DecCfg {
     static constexpr int LD = DH + 8; // padded row (elements): conflict-free fragment loads
-    static constexpr int SMEM = (2 * 128 * LD + 16 * LD) * 2 + 4 * 16 * DH * 4 + 2 * 4 * 16 * 4;
+    // K, V, Q tiles and the per-warp max / sum; the per-warp outputs [4][16][DH] fp32 reuse the K
+    // tile, which no warp reads after S (three CTAs fit per SM)
+    static constexpr int SMEM = (2 * 128 * LD + 16 * LD) * 2 + 2 * 4 * 16 * 4;
+    static_assert(4 * 16 * DH * 4 <= 128 * LD * 2, "output scratch fits in the K tile");
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
@@ -231,9 +234,9 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
     uint16_t* sK = reinterpret_cast<uint16_t*>(smem_raw);
     uint16_t* sV = sK + 128 * LD;
     uint16_t* sQ = sV + 128 * LD;
-    float* sO = reinterpret_cast<float*>(sQ + 16 * LD); // [4][16][DH]
-    float* sMax = sO + 4 * 16 * DH;                      // [4][16]
-    float* sSum = sMax + 4 * 16;                         // [4][16]
+    float* sO = reinterpret_cast<float*>(sK);                  // [4][16][DH], written after S
+    float* sMax = reinterpret_cast<float*>(sQ + 16 * LD);     // [4][16]
+    float* sSum = sMax + 4 * 16;                               // [4][16]
 
     const int beta = blockIdx.x, r = blockIdx.y, slot = blockIdx.z;
     const int G = a.H_q / a.H_kv;
