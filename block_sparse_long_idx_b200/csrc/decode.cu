@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(32) decode_topk_kernel(DecodeArgs a, int nb_ma
     const float* row = a.pooled + ((int64_t)beta * a.H_kv + r) * nb_max;
     TopkList list;
     list.init(a.k - 1);
-    for (int b = lane; b < local; b += 32) list.offer(row[b], b);
+    for (int b = lane; b < local; b += 32) list.offer_ascending(row[b], b); // each lane: ascending blocks
     float bv[kMaxK - 1];
     int bb[kMaxK - 1];
     warp_merge(list, a.k - 1, bv, bb);
