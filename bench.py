@@ -336,6 +336,32 @@ def gpu_arm(args, rank, world):
 
     pf_total, dec_total = replicas.max_over_ranks([sum(pf_ms), sum(dec_ms)], device=dev)
 
+    # the decode step captured once in a CUDA graph and replayed (how a serving loop would run it)
+    decode_graph = None
+    if dcfg:
+        cs = torch.cuda.Stream()
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs):
+            decode()
+        torch.cuda.current_stream().wait_stream(cs)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            decode()
+        for _ in range(args.warmup):
+            graph.replay()
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for st in range(args.steps):
+            flush.zero_()
+            gev[st][0].record()
+            graph.replay()
+            gev[st][1].record()
+        torch.cuda.synchronize()
+        (g_ms,) = replicas.max_over_ranks([sum(a.elapsed_time(b) for a, b in gev)], device=dev)
+        decode_graph = {"value": world * dcfg.B * args.steps / (g_ms / 1000.0), "unit": UNIT,
+                        "ms_per_step": g_ms / args.steps,
+                        "note": "the same decode step captured in a CUDA graph and replayed, L2 flushed before each"}
+        del graph
+
     # packed-batch (varlen) prefill of the same model shape: 16 sequences, 131072 tokens in total
     varlen = None
     if not args.no_varlen:
@@ -472,6 +498,7 @@ def gpu_arm(args, rank, world):
             "prefill_ms_per_step": pf_total / args.steps,
             "decode": ({"value": world * dcfg.B * args.steps / (dec_total / 1000.0), "unit": UNIT,
                         "ms_per_step": dec_total / args.steps} if dcfg else None),
+            "decode_graph": decode_graph,
             "roofline": roof, "kernels": kstats, "cpu_baseline": cpu_base, "e2e": e2e, "varlen": varlen,
             "gpu_launches": int(launches), "clocks": clocks.summary(), "wall_s_timed": wall}
     print(json.dumps(line), flush=True)
