@@ -174,3 +174,28 @@ def test_missing_library_fails_loudly(tmp_path):
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
                          cwd=str(tmp_path))
     assert "IMPORT_ERROR True" in out.stdout, out.stdout + out.stderr
+
+
+def test_varlen_workspace_sizes_follow_the_batch(msa):
+    """Workspace sizing of the packed-batch prefill: empty sequences are accepted, adding tokens or
+    cached prefixes never shrinks the workspace, and a batch of one sequence needs at least the
+    single-sequence prefill workspace."""
+    import numpy as np
+
+    lib = msa.lib
+    c_vp = ctypes.c_void_p
+
+    def size(cu, cuk=None, rows=0):
+        a = np.asarray(cu, dtype=np.int32)
+        b = None if cuk is None else np.asarray(cuk, dtype=np.int32)
+        return lib.msa_sparse_prefill_varlen_workspace_size(
+            a.ctypes.data_as(c_vp), None if b is None else b.ctypes.data_as(c_vp), len(cu) - 1, 16, 2, 128, 128, 8,
+            rows)
+
+    base = size([0, 1000, 3000])
+    assert base > 0
+    assert size([0, 0, 1000, 1000, 3000]) >= base > 0          # empty sequences
+    assert size([0, 1000, 5000]) > base                        # more tokens
+    assert size([0, 1000, 3000], [0, 1256, 3256]) >= base      # cached prefixes (256 each) add key blocks
+    single = lib.msa_sparse_prefill_workspace_size(3000, 16, 2, 128, 128, 8, 0, 1)
+    assert size([0, 3000]) >= single
