@@ -45,7 +45,8 @@ def parse_args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch (varlen) prefill leg")
     ap.add_argument("--decode-workload", default=synth.DECODE64.name, choices=sorted(synth.DECODE_CONFIGS))
-    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--e2e-steps", type=int, default=8,
+                    help="pipelined host-buffer steps (the first input copy and the last output copy are not overlapped)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-oracle sample time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows-per-pass", type=int, default=0, help="cap the prefill partial buffer (0 = whole N)")
