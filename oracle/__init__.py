@@ -1,4 +1,4 @@
-"""CPU oracle for the MSA forward path (test infrastructure only).
+"""CPU oracle for the MSA forward path and its backward (test infrastructure only).
 
 Only the tests, the package smoke check and the benchmark's CPU-baseline leg may import this
 package. It wraps the plain C99 + OpenMP oracle in ``msa_oracle.c`` with numpy marshalling.
@@ -57,8 +57,17 @@ class Oracle:
                                              _int, _c_i32p, _c_f64p, _c_f64p, _int]
         L.msa_oracle_decode.argtypes = [_c_u16p, _c_u16p, _c_u16p, _c_u16p, _c_u16p, _c_i32p, _int, _i64, _int, _int,
                                         _int, _int, _int, _int, _c_f64p, _c_f64p, _c_i32p, _int]
+        L.msa_oracle_backward_dq_rows.argtypes = [_c_u16p, _c_u16p, _c_i64p, _i64, _c_u16p, _c_u16p, _i64, _int, _int,
+                                                  _int, _int, _int, _c_i32p, _c_f64p, _int]
+        L.msa_oracle_backward_dkv_blocks.argtypes = [_c_u16p, _c_u16p, _c_u16p, _c_u16p, _i64, _int, _int, _int, _int,
+                                                     _int, _c_i32p, _c_i32p, _i64, _c_f64p, _c_f64p, _int]
+        L.msa_oracle_kl_rows.argtypes = [_c_u16p, _c_u16p, _c_i64p, _i64, _c_u16p, _c_u16p, _i64, _int, _int, _int,
+                                         _int, _int, _int, _c_i32p, ctypes.c_double, _c_f64p, _c_f64p, _int]
+        L.msa_oracle_kl_dk_idx_blocks.argtypes = [_c_u16p, _c_u16p, _c_u16p, _c_u16p, _i64, _int, _int, _int, _int,
+                                                  _int, _int, _c_i32p, _c_i32p, _i64, ctypes.c_double, _c_f64p, _int]
         for f in ("msa_oracle_select_rows", "msa_oracle_kv2q", "msa_oracle_attend_rows", "msa_oracle_decode",
-                  "msa_oracle_max_threads"):
+                  "msa_oracle_max_threads", "msa_oracle_backward_dq_rows", "msa_oracle_backward_dkv_blocks",
+                  "msa_oracle_kl_rows", "msa_oracle_kl_dk_idx_blocks"):
             getattr(L, f).restype = _int
         self.L = L
 
@@ -173,6 +182,81 @@ class Oracle:
             raise ValueError("msa_oracle_decode: bad arguments")
         return sel, out, lse
 
+    # ------------------------------------------------------------------ backward
+    def backward_dq_rows(self, q, dout, kk, v, rows, sel, B_k: int, n_threads: int = 0) -> np.ndarray:
+        """Main-branch dq of the given rows (selections sel [len(rows), H_kv, k] held fixed).
+
+        q, dout [N, H_q, d_h], kk/v [N, H_kv, d_h] bf16 bits. Returns f64 [len(rows), H_q, d_h]."""
+        N, H_kv, d_h = kk.shape
+        H_q = q.shape[1]
+        k = sel.shape[2]
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        qg, dg = _u16(q[rows]), _u16(dout[rows])
+        kc, vc = _u16(kk), _u16(v)
+        sel = np.ascontiguousarray(sel, dtype=np.int32)
+        dq = np.empty((len(rows), H_q, d_h), dtype=np.float64)
+        rc = self.L.msa_oracle_backward_dq_rows(_p(qg, _c_u16p), _p(dg, _c_u16p), _p(rows, _c_i64p), len(rows),
+                                                _p(kc, _c_u16p), _p(vc, _c_u16p), N, H_q, H_kv, d_h, B_k, k,
+                                                _p(sel, _c_i32p), _p(dq, _c_f64p), n_threads)
+        if rc:
+            raise ValueError("msa_oracle_backward_dq_rows: bad arguments")
+        return dq
+
+    def backward_dkv_blocks(self, q, dout, kk, v, sel, pairs, B_k: int, n_threads: int = 0):
+        """Main-branch dk, dv of whole KV blocks. sel [N, H_kv, k]: selections of every row;
+        pairs [(r, b), ...]. Returns (dk, dv) f64 [len(pairs), B_k, d_h] (rows past N are zero)."""
+        N, H_kv, d_h = kk.shape
+        H_q = q.shape[1]
+        k = sel.shape[2]
+        qc, dc, kc, vc = _u16(q), _u16(dout), _u16(kk), _u16(v)
+        sel = np.ascontiguousarray(sel, dtype=np.int32)
+        pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+        dk = np.empty((len(pr), B_k, d_h), dtype=np.float64)
+        dv = np.empty((len(pr), B_k, d_h), dtype=np.float64)
+        rc = self.L.msa_oracle_backward_dkv_blocks(_p(qc, _c_u16p), _p(dc, _c_u16p), _p(kc, _c_u16p), _p(vc, _c_u16p),
+                                                   N, H_q, H_kv, d_h, B_k, k, _p(sel, _c_i32p), _p(pr, _c_i32p),
+                                                   len(pr), _p(dk, _c_f64p), _p(dv, _c_f64p), n_threads)
+        if rc:
+            raise ValueError("msa_oracle_backward_dkv_blocks: bad arguments")
+        return dk, dv
+
+    def kl_rows(self, q, q_idx, kk, k_idx, rows, sel, B_k: int, w: float = 1.0, n_threads: int = 0):
+        """Index-branch KL of the given rows and its gradient in q_idx (scaled by w).
+
+        Returns (kl f64 [len(rows), H_kv], dq_idx f64 [len(rows), H_kv, d_idx])."""
+        N, H_kv, d_h = kk.shape
+        H_q, d_idx = q.shape[1], k_idx.shape[2]
+        k = sel.shape[2]
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        qg, qig = _u16(q[rows]), _u16(q_idx[rows])
+        kc, kic = _u16(kk), _u16(k_idx)
+        sel = np.ascontiguousarray(sel, dtype=np.int32)
+        kl = np.empty((len(rows), H_kv), dtype=np.float64)
+        dq_idx = np.empty((len(rows), H_kv, d_idx), dtype=np.float64)
+        rc = self.L.msa_oracle_kl_rows(_p(qg, _c_u16p), _p(qig, _c_u16p), _p(rows, _c_i64p), len(rows), _p(kc, _c_u16p),
+                                       _p(kic, _c_u16p), N, H_q, H_kv, d_h, d_idx, B_k, k, _p(sel, _c_i32p), float(w),
+                                       _p(kl, _c_f64p), _p(dq_idx, _c_f64p), n_threads)
+        if rc:
+            raise ValueError("msa_oracle_kl_rows: bad arguments")
+        return kl, dq_idx
+
+    def kl_dk_idx_blocks(self, q, q_idx, kk, k_idx, sel, pairs, B_k: int, w: float = 1.0, n_threads: int = 0):
+        """Gradient of the index-branch KL in k_idx for whole KV blocks (scaled by w).
+        sel [N, H_kv, k]: selections of every row. Returns f64 [len(pairs), B_k, d_idx]."""
+        N, H_kv, d_h = kk.shape
+        H_q, d_idx = q.shape[1], k_idx.shape[2]
+        k = sel.shape[2]
+        qc, qic, kc, kic = _u16(q), _u16(q_idx), _u16(kk), _u16(k_idx)
+        sel = np.ascontiguousarray(sel, dtype=np.int32)
+        pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+        g = np.empty((len(pr), B_k, d_idx), dtype=np.float64)
+        rc = self.L.msa_oracle_kl_dk_idx_blocks(_p(qc, _c_u16p), _p(qic, _c_u16p), _p(kc, _c_u16p), _p(kic, _c_u16p), N,
+                                                H_q, H_kv, d_h, d_idx, B_k, k, _p(sel, _c_i32p), _p(pr, _c_i32p),
+                                                len(pr), float(w), _p(g, _c_f64p), n_threads)
+        if rc:
+            raise ValueError("msa_oracle_kl_dk_idx_blocks: bad arguments")
+        return g
+
 
 _default = None
 
@@ -210,6 +294,22 @@ def prefill_varlen_rows(*a, **kw):
 
 def decode(*a, **kw):
     return default().decode(*a, **kw)
+
+
+def backward_dq_rows(*a, **kw):
+    return default().backward_dq_rows(*a, **kw)
+
+
+def backward_dkv_blocks(*a, **kw):
+    return default().backward_dkv_blocks(*a, **kw)
+
+
+def kl_rows(*a, **kw):
+    return default().kl_rows(*a, **kw)
+
+
+def kl_dk_idx_blocks(*a, **kw):
+    return default().kl_dk_idx_blocks(*a, **kw)
 
 
 def max_threads() -> int:

@@ -1,5 +1,6 @@
 /*
- * msa_oracle.c -- plain CPU oracle for the MiniMax Sparse Attention (MSA) forward path.
+ * msa_oracle.c -- plain CPU oracle for the MiniMax Sparse Attention (MSA) forward path and its
+ * backward (gradients of the main branch, KL training signal of the index branch).
  *
  * TEST INFRASTRUCTURE ONLY. Nothing in the product path may call, link or load this file;
  * only the tests, the package's smoke check and the benchmark's CPU-baseline leg use it.
@@ -25,6 +26,8 @@
  *      q_h . k_j / sqrt(d_h); out = sum_j p_j v_j; lse = max + log(sum exp(. - max)) in the
  *      units of the scaled logits.
  *  (4) Decode: (1)+(3) for the single query at position len-1 of each cached sequence.
+ *  (5) Main Branch backward: the gradient of (3) in q, k and v with the selected sets fixed.
+ *  (6) Index Branch KL alignment loss (explainer section 03) and its gradient in q_idx, k_idx.
  *
  * Inputs are bf16 bit patterns widened exactly to double. All sums are in double.
  */
@@ -320,4 +323,366 @@ int msa_oracle_decode(const uint16_t* q, const uint16_t* q_idx, const uint16_t* 
         if (rc) return rc;
     }
     return 0;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* (5) Main Branch backward: the gradient of (3) with the selected sets held fixed.          */
+/* ---------------------------------------------------------------------------------------- */
+/*
+ * The Top-k selection is not differentiable (explainer section 03), so the language-model loss
+ * reaches q, k and v only through the exact softmax attention over T(i, r) of (3). For one
+ * (row i, head h) with p_j = exp(q.k_j*scale - lse), out = sum_j p_j v_j and upstream dout:
+ *   D      = dout . out
+ *   ds_j   = p_j * (dout . v_j - D)          (softmax Jacobian applied to dout . v_j)
+ *   dq_i  += scale * sum_j ds_j k_j
+ *   dk_j  += scale * ds_j q_i
+ *   dv_j  += p_j dout
+ * lse and out are recomputed here from q, k, v (the forward pass stores them; the backward of
+ * the explainer's kernels reads them back, section 05-2, "LSE fusion" paragraph).
+ */
+
+/* logits and weights of (i, h) over T in the order of the selected blocks; returns |T|.
+ * tok[n] = key position of logits[n]. */
+static int64_t probs_one(const double* q, const uint16_t* kseq, int64_t i, int r, int H_kv, int d_h, int B_k, int k,
+                         const int32_t* sel, double* p, int64_t* tok)
+{
+    const double scale = 1.0 / sqrt((double)d_h);
+    int64_t n = 0;
+    double m = -INFINITY;
+    for (int s = 0; s < k; ++s) {
+        int32_t b = sel[s];
+        if (b < 0) continue;
+        for (int64_t j = (int64_t)b * B_k; j < ((int64_t)b + 1) * B_k && j <= i; ++j) {
+            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;
+            double dot = 0.0;
+            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);
+            p[n] = dot * scale;
+            tok[n] = j;
+            if (p[n] > m) m = p[n];
+            ++n;
+        }
+    }
+    double z = 0.0;
+    for (int64_t t = 0; t < n; ++t) {
+        p[t] = exp(p[t] - m);
+        z += p[t];
+    }
+    for (int64_t t = 0; t < n; ++t) p[t] /= z;
+    return n;
+}
+
+/* ds_j of (i, h) over T (in place of p), given p and dout; returns D = dout . out. */
+static double dscores_one(const double* dout, const uint16_t* vseq, int r, int H_kv, int d_h, int64_t n,
+                          const int64_t* tok, const double* p, double* ds)
+{
+    double out[512];
+    for (int d = 0; d < d_h; ++d) out[d] = 0.0;
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t* vr = vseq + ((size_t)tok[t] * H_kv + r) * d_h;
+        for (int d = 0; d < d_h; ++d) out[d] += p[t] * bf16_to_double(vr[d]);
+    }
+    double D = 0.0;
+    for (int d = 0; d < d_h; ++d) D += dout[d] * out[d];
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t* vr = vseq + ((size_t)tok[t] * H_kv + r) * d_h;
+        double dp = 0.0;
+        for (int d = 0; d < d_h; ++d) dp += dout[d] * bf16_to_double(vr[d]);
+        ds[t] = p[t] * (dp - D);
+    }
+    return D;
+}
+
+/*
+ * dq of requested rows.
+ *   q, dout : [n_rows, H_q, d_h] bf16, gathered for the requested rows
+ *   rows    : [n_rows] positions;  kk, v : [N, H_kv, d_h] bf16
+ *   sel     : [n_rows, H_kv, k] int32 selections of the rows
+ *   dq      : [n_rows, H_q, d_h] double
+ */
+int msa_oracle_backward_dq_rows(const uint16_t* q, const uint16_t* dout, const int64_t* rows, int64_t n_rows,
+                                const uint16_t* kk, const uint16_t* v, int64_t N, int H_q, int H_kv, int d_h,
+                                int B_k, int k, const int32_t* sel, double* dq, int n_threads)
+{
+    if (!q || !dout || !rows || !kk || !v || !sel || !dq || H_kv < 1 || H_q % H_kv || d_h < 1 || d_h > 512)
+        return -1;
+    for (int64_t t = 0; t < n_rows; ++t)
+        if (rows[t] < 0 || rows[t] >= N) return -1;
+    const int G = H_q / H_kv;
+    const double scale = 1.0 / sqrt((double)d_h);
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        double* p = (double*)malloc(sizeof(double) * (size_t)k * B_k);
+        double* ds = (double*)malloc(sizeof(double) * (size_t)k * B_k);
+        int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)k * B_k);
+        const int ok = p && ds && tok;
+        if (!ok) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1) collapse(2)
+        for (int64_t t = 0; t < n_rows; ++t)
+            for (int h = 0; h < H_q; ++h)
+                if (ok) {
+                    const int r = h / G;
+                    double qd[512], dod[512];
+                    for (int d = 0; d < d_h; ++d) {
+                        qd[d] = bf16_to_double(q[((size_t)t * H_q + h) * d_h + d]);
+                        dod[d] = bf16_to_double(dout[((size_t)t * H_q + h) * d_h + d]);
+                    }
+                    const int32_t* s_r = sel + ((size_t)t * H_kv + r) * k;
+                    const int64_t n = probs_one(qd, kk, rows[t], r, H_kv, d_h, B_k, k, s_r, p, tok);
+                    dscores_one(dod, v, r, H_kv, d_h, n, tok, p, ds);
+                    double* g = dq + ((size_t)t * H_q + h) * d_h;
+                    for (int d = 0; d < d_h; ++d) g[d] = 0.0;
+                    for (int64_t u = 0; u < n; ++u) {
+                        const uint16_t* kr = kk + ((size_t)tok[u] * H_kv + r) * d_h;
+                        for (int d = 0; d < d_h; ++d) g[d] += scale * ds[u] * bf16_to_double(kr[d]);
+                    }
+                }
+        free(p);
+        free(ds);
+        free(tok);
+    }
+    return err;
+}
+
+/* does (i, r) select block b? */
+static int selects(const int32_t* s_ir, int k, int32_t b)
+{
+    for (int s = 0; s < k; ++s)
+        if (s_ir[s] == b) return 1;
+    return 0;
+}
+
+/*
+ * dk and dv of whole KV blocks: for each requested (group r, block b), every row i whose set
+ * contains b and every head h of group r contribute to the keys j <= i of block b.
+ *   q, dout : [N, H_q, d_h] bf16 (all rows);  kk, v : [N, H_kv, d_h] bf16
+ *   sel     : [N, H_kv, k] int32 selections of all rows
+ *   pairs   : [n_pairs, 2] (r, b)
+ *   dk, dv  : [n_pairs, B_k, d_h] double (rows past N are zero)
+ */
+int msa_oracle_backward_dkv_blocks(const uint16_t* q, const uint16_t* dout, const uint16_t* kk, const uint16_t* v,
+                                   int64_t N, int H_q, int H_kv, int d_h, int B_k, int k, const int32_t* sel,
+                                   const int32_t* pairs, int64_t n_pairs, double* dk, double* dv, int n_threads)
+{
+    if (!q || !dout || !kk || !v || !sel || !pairs || !dk || !dv || H_kv < 1 || H_q % H_kv || d_h < 1 ||
+        d_h > 512)
+        return -1;
+    const int64_t nb = (N + B_k - 1) / B_k;
+    for (int64_t t = 0; t < n_pairs; ++t)
+        if (pairs[2 * t] < 0 || pairs[2 * t] >= H_kv || pairs[2 * t + 1] < 0 || pairs[2 * t + 1] >= nb) return -1;
+    const int G = H_q / H_kv;
+    const double scale = 1.0 / sqrt((double)d_h);
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        double* p = (double*)malloc(sizeof(double) * (size_t)k * B_k);
+        double* ds = (double*)malloc(sizeof(double) * (size_t)k * B_k);
+        int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)k * B_k);
+        const int ok = p && ds && tok;
+        if (!ok) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < n_pairs; ++t) {
+            if (!ok) continue;
+            const int r = pairs[2 * t];
+            const int32_t b = pairs[2 * t + 1];
+            double* gk = dk + (size_t)t * B_k * d_h;
+            double* gv = dv + (size_t)t * B_k * d_h;
+            for (int64_t x = 0; x < (int64_t)B_k * d_h; ++x) gk[x] = gv[x] = 0.0;
+            for (int64_t i = (int64_t)b * B_k; i < N; ++i) {
+                const int32_t* s_ir = sel + ((size_t)i * H_kv + r) * k;
+                if (!selects(s_ir, k, b)) continue;
+                for (int h = r * G; h < (r + 1) * G; ++h) {
+                    double qd[512], dod[512];
+                    for (int d = 0; d < d_h; ++d) {
+                        qd[d] = bf16_to_double(q[((size_t)i * H_q + h) * d_h + d]);
+                        dod[d] = bf16_to_double(dout[((size_t)i * H_q + h) * d_h + d]);
+                    }
+                    const int64_t n = probs_one(qd, kk, i, r, H_kv, d_h, B_k, k, s_ir, p, tok);
+                    dscores_one(dod, v, r, H_kv, d_h, n, tok, p, ds);
+                    for (int64_t u = 0; u < n; ++u) {
+                        if (tok[u] / B_k != b) continue;
+                        const int64_t jj = tok[u] - (int64_t)b * B_k;
+                        for (int d = 0; d < d_h; ++d) {
+                            gk[jj * d_h + d] += scale * ds[u] * qd[d];
+                            gv[jj * d_h + d] += p[u] * dod[d];
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(ds);
+        free(tok);
+    }
+    return err;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* (6) Index Branch training signal: the KL alignment loss and its gradient.                 */
+/* ---------------------------------------------------------------------------------------- */
+/*
+ * Explainer section 03 ("KL Loss"): for query i and group r, over the token set T(i, r) of the
+ * selected blocks,
+ *   student  P_idx_j = softmax_T(s_idx)_j,   s_idx_j = q_idx[i,r] . k_idx[j,r]   (the index score
+ *            of (1), unscaled: the pages give the index score no scale)
+ *   teacher  P_j = (1/G) sum_{h in group r} p_{h,j}     (the G heads' attention weights of (3),
+ *            averaged as probabilities)
+ *   KL(i, r) = sum_j P_j (log P_j - log P_idx_j)
+ * The loss averages KL over positions and groups; the teacher is stop-gradient, so the gradient
+ * reaches only the index projections: dKL/ds_idx_j = P_idx_j - P_j, hence
+ *   dq_idx[i,r] += w * sum_j (P_idx_j - P_j) k_idx[j,r]
+ *   dk_idx[j,r] += w * (P_idx_j - P_j) q_idx[i,r]
+ * with w the caller's weight (1 / (rows * H_kv) for the mean).
+ */
+
+/* teacher weights P over T of (i, r) into P[0..n), with tok[]; student log-weights into lq[]. */
+static int64_t kl_dists(const uint16_t* q_i /*[H_q, d_h]*/, const uint16_t* qidx_ir, const uint16_t* kk,
+                        const uint16_t* k_idx, int64_t i, int r, int H_q, int H_kv, int d_h, int d_idx, int B_k, int k,
+                        const int32_t* s_ir, double* P, double* lq, double* p, int64_t* tok)
+{
+    const int G = H_q / H_kv;
+    int64_t n = 0;
+    for (int h = r * G; h < (r + 1) * G; ++h) {
+        double qd[512];
+        for (int d = 0; d < d_h; ++d) qd[d] = bf16_to_double(q_i[(size_t)h * d_h + d]);
+        n = probs_one(qd, kk, i, r, H_kv, d_h, B_k, k, s_ir, p, tok);
+        for (int64_t t = 0; t < n; ++t) P[t] = (h == r * G ? 0.0 : P[t]) + p[t] / G;
+    }
+    double m = -INFINITY;
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t* kr = k_idx + ((size_t)tok[t] * H_kv + r) * d_idx;
+        double s = 0.0;
+        for (int d = 0; d < d_idx; ++d) s += bf16_to_double(qidx_ir[d]) * bf16_to_double(kr[d]);
+        lq[t] = s;
+        if (s > m) m = s;
+    }
+    double z = 0.0;
+    for (int64_t t = 0; t < n; ++t) z += exp(lq[t] - m);
+    const double lz = m + log(z);
+    for (int64_t t = 0; t < n; ++t) lq[t] -= lz;
+    return n;
+}
+
+/*
+ * KL(i, r) and dq_idx of requested rows.
+ *   q      : [n_rows, H_q, d_h] bf16;  q_idx : [n_rows, H_kv, d_idx] bf16 (gathered rows)
+ *   kk     : [N, H_kv, d_h] bf16;      k_idx : [N, H_kv, d_idx] bf16
+ *   sel    : [n_rows, H_kv, k] int32
+ *   kl     : [n_rows, H_kv] double;    dq_idx : [n_rows, H_kv, d_idx] double (scaled by w)
+ */
+int msa_oracle_kl_rows(const uint16_t* q, const uint16_t* q_idx, const int64_t* rows, int64_t n_rows,
+                       const uint16_t* kk, const uint16_t* k_idx, int64_t N, int H_q, int H_kv, int d_h, int d_idx,
+                       int B_k, int k, const int32_t* sel, double w, double* kl, double* dq_idx, int n_threads)
+{
+    if (!q || !q_idx || !rows || !kk || !k_idx || !sel || !kl || !dq_idx || H_kv < 1 || H_q % H_kv || d_h < 1 ||
+        d_h > 512 || d_idx < 1)
+        return -1;
+    for (int64_t t = 0; t < n_rows; ++t)
+        if (rows[t] < 0 || rows[t] >= N) return -1;
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        const size_t cap = (size_t)k * B_k;
+        double* P = (double*)malloc(sizeof(double) * cap);
+        double* lq = (double*)malloc(sizeof(double) * cap);
+        double* p = (double*)malloc(sizeof(double) * cap);
+        int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * cap);
+        const int ok = P && lq && p && tok;
+        if (!ok) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1) collapse(2)
+        for (int64_t t = 0; t < n_rows; ++t)
+            for (int r = 0; r < H_kv; ++r)
+                if (ok) {
+                    const uint16_t* qi = q_idx + ((size_t)t * H_kv + r) * d_idx;
+                    const int64_t n = kl_dists(q + (size_t)t * H_q * d_h, qi, kk, k_idx, rows[t], r, H_q, H_kv, d_h,
+                                               d_idx, B_k, k, sel + ((size_t)t * H_kv + r) * k, P, lq, p, tok);
+                    double acc = 0.0;
+                    double* g = dq_idx + ((size_t)t * H_kv + r) * d_idx;
+                    for (int d = 0; d < d_idx; ++d) g[d] = 0.0;
+                    for (int64_t u = 0; u < n; ++u) {
+                        acc += P[u] * (log(P[u]) - lq[u]);
+                        const double gs = w * (exp(lq[u]) - P[u]);
+                        const uint16_t* kr = k_idx + ((size_t)tok[u] * H_kv + r) * d_idx;
+                        for (int d = 0; d < d_idx; ++d) g[d] += gs * bf16_to_double(kr[d]);
+                    }
+                    kl[(size_t)t * H_kv + r] = acc;
+                }
+        free(P);
+        free(lq);
+        free(p);
+        free(tok);
+    }
+    return err;
+}
+
+/*
+ * dk_idx of whole KV blocks: every row i whose set of group r contains b contributes to the keys
+ * j <= i of block b.
+ *   q : [N, H_q, d_h], q_idx : [N, H_kv, d_idx], kk : [N, H_kv, d_h], k_idx : [N, H_kv, d_idx] (bf16)
+ *   sel : [N, H_kv, k] int32;  pairs : [n_pairs, 2] (r, b)
+ *   dk_idx : [n_pairs, B_k, d_idx] double (scaled by w; rows past N are zero)
+ */
+int msa_oracle_kl_dk_idx_blocks(const uint16_t* q, const uint16_t* q_idx, const uint16_t* kk, const uint16_t* k_idx,
+                                int64_t N, int H_q, int H_kv, int d_h, int d_idx, int B_k, int k, const int32_t* sel,
+                                const int32_t* pairs, int64_t n_pairs, double w, double* dk_idx, int n_threads)
+{
+    if (!q || !q_idx || !kk || !k_idx || !sel || !pairs || !dk_idx || H_kv < 1 || H_q % H_kv || d_h < 1 ||
+        d_h > 512 || d_idx < 1)
+        return -1;
+    const int64_t nb = (N + B_k - 1) / B_k;
+    for (int64_t t = 0; t < n_pairs; ++t)
+        if (pairs[2 * t] < 0 || pairs[2 * t] >= H_kv || pairs[2 * t + 1] < 0 || pairs[2 * t + 1] >= nb) return -1;
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        const size_t cap = (size_t)k * B_k;
+        double* P = (double*)malloc(sizeof(double) * cap);
+        double* lq = (double*)malloc(sizeof(double) * cap);
+        double* p = (double*)malloc(sizeof(double) * cap);
+        int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * cap);
+        const int ok = P && lq && p && tok;
+        if (!ok) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < n_pairs; ++t) {
+            if (!ok) continue;
+            const int r = pairs[2 * t];
+            const int32_t b = pairs[2 * t + 1];
+            double* g = dk_idx + (size_t)t * B_k * d_idx;
+            for (int64_t x = 0; x < (int64_t)B_k * d_idx; ++x) g[x] = 0.0;
+            for (int64_t i = (int64_t)b * B_k; i < N; ++i) {
+                const int32_t* s_ir = sel + ((size_t)i * H_kv + r) * k;
+                if (!selects(s_ir, k, b)) continue;
+                const uint16_t* qi = q_idx + ((size_t)i * H_kv + r) * d_idx;
+                const int64_t n = kl_dists(q + (size_t)i * H_q * d_h, qi, kk, k_idx, i, r, H_q, H_kv, d_h, d_idx, B_k,
+                                           k, s_ir, P, lq, p, tok);
+                for (int64_t u = 0; u < n; ++u) {
+                    if (tok[u] / B_k != b) continue;
+                    const int64_t jj = tok[u] - (int64_t)b * B_k;
+                    const double gs = w * (exp(lq[u]) - P[u]);
+                    for (int d = 0; d < d_idx; ++d) g[jj * d_idx + d] += gs * bf16_to_double(qi[d]);
+                }
+            }
+        }
+        free(P);
+        free(lq);
+        free(p);
+        free(tok);
+    }
+    return err;
 }

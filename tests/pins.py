@@ -14,6 +14,7 @@ import math
 import numpy as np
 
 from block_sparse_long_idx_b200.synth import bf16_bits_to_f64, f32_to_bf16_bits, int_uniform_bf16, normal_bf16
+from tests import ref_autograd
 from tests import ref_numpy as ref
 
 # (N, H_q, H_kv, d_h, d_idx, B_k, k) -- small shapes spanning several blocks, ragged tails, k larger
@@ -296,6 +297,114 @@ def check_varlen_cached_prefix_matches_dense(o):
         assert np.max(np.abs(lse[lo:hi] - want_lse[prefix[s]:])) < 1e-12, s
 
 
+# ------------------------------------------------------------------------------------ backward
+
+def _bwd_case(o, N, H_q, H_kv, d_h, d_idx, B_k, k, seed):
+    inp = _attn_inputs(N, H_q, H_kv, d_h, d_idx, seed)
+    inp["dout"] = normal_bf16((N, H_q, d_h), seed, "ado")
+    sel = o.select_rows(inp["q_idx"], inp["k_idx"], np.arange(N), B_k, k)  # [N, H_kv, k]
+    nb = (N + B_k - 1) // B_k
+    pairs = [(r, b) for r in range(H_kv) for b in range(nb)]
+    return inp, sel, pairs, nb
+
+
+def _blocks_to_tokens(g, H_kv, nb, B_k, N):
+    """[(r, b) pairs in r-major order, B_k, d] -> [N, H_kv, d]."""
+    d = g.shape[-1]
+    return g.reshape(H_kv, nb * B_k, d)[:, :N].transpose(1, 0, 2)
+
+
+BWD_SHAPES = [(96, 4, 2, 16, 8, 16, 3), (70, 2, 1, 8, 8, 8, 4), (64, 4, 2, 16, 8, 16, 4)]  # last: k*B_k >= N
+
+
+def check_backward_autograd(o):
+    """Main-branch dq, dk, dv equal autograd of masked dense attention under the selection mask."""
+    for (N, H_q, H_kv, d_h, d_idx, B_k, k) in BWD_SHAPES:
+        inp, sel, pairs, nb = _bwd_case(o, N, H_q, H_kv, d_h, d_idx, B_k, k, N + 11)
+        dq = o.backward_dq_rows(inp["q"], inp["dout"], inp["k"], inp["v"], np.arange(N), sel, B_k)
+        dk, dv = o.backward_dkv_blocks(inp["q"], inp["dout"], inp["k"], inp["v"], sel, pairs, B_k)
+        allowed = ref.selection_mask(np.ascontiguousarray(sel.transpose(1, 0, 2)), N, B_k)
+        wq, wk, wv = ref_autograd.attention_grads(inp["q"], inp["k"], inp["v"], inp["dout"], allowed)
+        assert np.max(np.abs(dq - wq)) < 1e-10, np.max(np.abs(dq - wq))
+        assert np.max(np.abs(_blocks_to_tokens(dk, H_kv, nb, B_k, N) - wk)) < 1e-10
+        assert np.max(np.abs(_blocks_to_tokens(dv, H_kv, nb, B_k, N) - wv)) < 1e-10
+        pad = nb * B_k - N
+        if pad:
+            assert not np.any(dk.reshape(H_kv, nb * B_k, -1)[:, N:]) and not np.any(dv.reshape(H_kv, nb * B_k, -1)[:, N:])
+
+
+def check_backward_identical_keys(o):
+    """All keys equal: every logit of a row is the same constant direction, so the softmax Jacobian
+    annihilates dq (sum_j ds_j = 0) while dv is the mean of dout over the rows that see each key."""
+    N, H_q, H_kv, d_h, d_idx, B_k, k = 80, 4, 2, 8, 8, 16, 3
+    inp, sel, pairs, nb = _bwd_case(o, N, H_q, H_kv, d_h, d_idx, B_k, k, 21)
+    inp["k"] = np.broadcast_to(inp["k"][:1], inp["k"].shape).copy()
+    dq = o.backward_dq_rows(inp["q"], inp["dout"], inp["k"], inp["v"], np.arange(N), sel, B_k)
+    assert np.max(np.abs(dq)) < 1e-12
+    _, dv = o.backward_dkv_blocks(inp["q"], inp["dout"], inp["k"], inp["v"], sel, pairs, B_k)
+    dv = _blocks_to_tokens(dv, H_kv, nb, B_k, N)
+    allowed = ref.selection_mask(np.ascontiguousarray(sel.transpose(1, 0, 2)), N, B_k)
+    dO = bf16_bits_to_f64(inp["dout"])
+    G = H_q // H_kv
+    for r in range(H_kv):
+        wts = allowed[r] / allowed[r].sum(axis=1, keepdims=True)  # uniform weights over T(i, r)
+        want = wts.T @ dO[:, r * G:(r + 1) * G, :].sum(axis=1)
+        assert np.max(np.abs(dv[:, r] - want)) < 1e-12
+
+
+def check_backward_dv_sums_to_dout(o):
+    """Attention weights of a row sum to one, so sum_j dv[j, r] = sum_i sum_{h in r} dout[i, h]."""
+    N, H_q, H_kv, d_h, d_idx, B_k, k = 150, 4, 2, 8, 8, 16, 4
+    inp, sel, pairs, nb = _bwd_case(o, N, H_q, H_kv, d_h, d_idx, B_k, k, 22)
+    _, dv = o.backward_dkv_blocks(inp["q"], inp["dout"], inp["k"], inp["v"], sel, pairs, B_k)
+    dv = _blocks_to_tokens(dv, H_kv, nb, B_k, N)
+    dO = bf16_bits_to_f64(inp["dout"])
+    G = H_q // H_kv
+    for r in range(H_kv):
+        assert np.max(np.abs(dv[:, r].sum(axis=0) - dO[:, r * G:(r + 1) * G].sum(axis=(0, 1)))) < 1e-10
+
+
+def check_kl_autograd(o):
+    """Index-branch KL per (row, group) and its gradients equal autograd of the KL loss (teacher
+    detached), with the loss weight 1/(N * H_kv) of the mean."""
+    for (N, H_q, H_kv, d_h, d_idx, B_k, k) in BWD_SHAPES:
+        inp, sel, pairs, nb = _bwd_case(o, N, H_q, H_kv, d_h, d_idx, B_k, k, N + 12)
+        inp["q_idx"] = normal_bf16(inp["q_idx"].shape, N, "klq")  # non-integer index scores
+        inp["k_idx"] = normal_bf16(inp["k_idx"].shape, N, "klk")
+        sel = o.select_rows(inp["q_idx"], inp["k_idx"], np.arange(N), B_k, k)
+        w = 1.0 / (N * H_kv)
+        kl, dqi = o.kl_rows(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], np.arange(N), sel, B_k, w)
+        dki = o.kl_dk_idx_blocks(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], sel, pairs, B_k, w)
+        allowed = ref.selection_mask(np.ascontiguousarray(sel.transpose(1, 0, 2)), N, B_k)
+        wkl, wq, wk = ref_autograd.kl_loss_grads(inp["q"], inp["k"], inp["q_idx"], inp["k_idx"], allowed, w)
+        assert np.max(np.abs(kl - wkl)) < 1e-10, np.max(np.abs(kl - wkl))
+        assert np.all(kl > -1e-12)  # Gibbs' inequality
+        assert np.max(np.abs(dqi - wq)) < 1e-12, np.max(np.abs(dqi - wq))
+        assert np.max(np.abs(_blocks_to_tokens(dki, H_kv, nb, B_k, N) - wk)) < 1e-12
+
+
+def check_kl_uniform_teacher_closed_form(o):
+    """q == 0 makes the teacher uniform over T, so KL(U || softmax(s)) = logsumexp(s) - mean(s) - log|T|
+    and dKL/ds = softmax(s) - 1/|T|; with q_idx == 0 as well the KL and its gradients vanish."""
+    N, H_q, H_kv, d_h, d_idx, B_k, k = 72, 4, 2, 8, 8, 8, 3
+    inp, sel, pairs, nb = _bwd_case(o, N, H_q, H_kv, d_h, d_idx, B_k, k, 23)
+    inp["q"] = np.zeros_like(inp["q"])
+    kl, dqi = o.kl_rows(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], np.arange(N), sel, B_k)
+    Qi, Ki = bf16_bits_to_f64(inp["q_idx"]), bf16_bits_to_f64(inp["k_idx"])
+    for i in range(0, N, 7):
+        for r in range(H_kv):
+            toks = [j for b in sel[i, r] if b >= 0 for j in range(b * B_k, min((b + 1) * B_k, i + 1))]
+            s = Ki[toks, r] @ Qi[i, r]
+            lse = s.max() + math.log(np.exp(s - s.max()).sum())
+            assert abs(kl[i, r] - (lse - s.mean() - math.log(len(toks)))) < 1e-10
+            g = np.exp(s - lse) - 1.0 / len(toks)
+            assert np.max(np.abs(dqi[i, r] - g @ Ki[toks, r])) < 1e-10
+    inp["q_idx"] = np.zeros_like(inp["q_idx"])
+    kl, dqi = o.kl_rows(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], np.arange(N), sel, B_k)
+    dki = o.kl_dk_idx_blocks(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], sel, pairs, B_k)
+    assert np.max(np.abs(kl)) < 1e-14 and np.max(np.abs(dqi)) < 1e-14 and np.max(np.abs(dki)) < 1e-14
+
+
 ALL_CHECKS = [
     check_selection_bruteforce,
     check_selection_ties_closed_form,
@@ -311,4 +420,9 @@ ALL_CHECKS = [
     check_decode_matches_prefill_row,
     check_varlen_matches_dense_per_sequence,
     check_varlen_cached_prefix_matches_dense,
+    check_backward_autograd,
+    check_backward_identical_keys,
+    check_backward_dv_sums_to_dout,
+    check_kl_autograd,
+    check_kl_uniform_teacher_closed_form,
 ]

@@ -32,16 +32,34 @@ MUTANTS = [
     ("tie_break_to_higher_block", "return (x->block > y->block) - (x->block < y->block);",
      "return (x->block < y->block) - (x->block > y->block);"),
     ("local_block_not_forced", "sel[n++] = (int32_t)local;", "if (take < k) sel[n++] = (int32_t)(local > 0 ? local - 1 : 0);"),
-    ("scale_1_over_d", "const double scale = 1.0 / sqrt((double)d_h);", "const double scale = 1.0 / (double)d_h;"),
-    ("causal_strict", "j < ((int64_t)b + 1) * B_k && j <= i; ++j) {\n            const uint16_t* kr",
-     "j < ((int64_t)b + 1) * B_k && j < i; ++j) {\n            const uint16_t* kr"),
+    ("scale_1_over_d", "const double scale = 1.0 / sqrt((double)d_h);\n    double q[512];",
+     "const double scale = 1.0 / (double)d_h;\n    double q[512];"),
+    ("bwd_logits_scale_1_over_d", "const double scale = 1.0 / sqrt((double)d_h);\n    int64_t n = 0;",
+     "const double scale = 1.0 / (double)d_h;\n    int64_t n = 0;"),
+    ("causal_strict", "j <= i; ++j) {\n            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;\n            double dot = 0.0;\n            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);\n            logits[n]",
+     "j < i; ++j) {\n            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;\n            double dot = 0.0;\n            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);\n            logits[n]"),
+    ("bwd_causal_strict", "j <= i; ++j) {\n            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;\n            double dot = 0.0;\n            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);\n            p[n]",
+     "j < i; ++j) {\n            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;\n            double dot = 0.0;\n            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);\n            p[n]"),
     ("pool_sum_not_max", "if (s > best) best = s; /* block max pooling */",
      "best = (best == -INFINITY ? 0.0 : best) + s;"),
     ("k_not_counting_local", "(int64_t)(k - 1);\n    for (int64_t t = 0; t < take",
      "(int64_t)(k);\n    for (int64_t t = 0; t < take"),
-    ("wrong_gqa_group", "const int r = h / G;", "const int r = h % H_kv;"),
+    ("wrong_gqa_group", "const int r = h / G;\n                    attend_one(",
+     "const int r = h % H_kv;\n                    attend_one("),
+    ("bwd_wrong_gqa_group", "const int r = h / G;\n                    double qd[512], dod[512];",
+     "const int r = h % H_kv;\n                    double qd[512], dod[512];"),
     ("lse_missing_max", "*lse = m + log(z);", "*lse = log(z);"),
     ("kv2q_slot_off_by_one", "ent[fill[b]++] = (int32_t)(i * k + s);", "ent[fill[b]++] = (int32_t)(i * k + s + 1);"),
+    ("bwd_softmax_jacobian_without_D", "ds[t] = p[t] * (dp - D);", "ds[t] = p[t] * dp;"),
+    ("bwd_dk_from_dout", "gk[jj * d_h + d] += scale * ds[u] * qd[d];", "gk[jj * d_h + d] += scale * ds[u] * dod[d];"),
+    ("bwd_dv_unweighted", "gv[jj * d_h + d] += p[u] * dod[d];", "gv[jj * d_h + d] += dod[d];"),
+    ("bwd_dq_unscaled", "for (int d = 0; d < d_h; ++d) g[d] += scale * ds[u] * bf16_to_double(kr[d]);",
+     "for (int d = 0; d < d_h; ++d) g[d] += ds[u] * bf16_to_double(kr[d]);"),
+    ("kl_teacher_summed_not_averaged", "P[t] = (h == r * G ? 0.0 : P[t]) + p[t] / G;",
+     "P[t] = (h == r * G ? 0.0 : P[t]) + p[t];"),
+    ("kl_gradient_sign", "const double gs = w * (exp(lq[u]) - P[u]);\n                        const uint16_t* kr",
+     "const double gs = w * (P[u] - exp(lq[u]));\n                        const uint16_t* kr"),
+    ("kl_student_scaled", "lq[t] = s;\n", "lq[t] = s / sqrt((double)d_idx);\n"),
 ]
 
 
