@@ -44,6 +44,7 @@ def parse_args():
     ap.add_argument("--workload", default=synth.P128K.name, choices=sorted(synth.PREFILL_CONFIGS))
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch (varlen) prefill leg")
+    ap.add_argument("--no-backward", action="store_true", help="skip the main-branch backward leg")
     ap.add_argument("--decode-workload", default=synth.DECODE64.name, choices=sorted(synth.DECODE_CONFIGS))
     ap.add_argument("--e2e-steps", type=int, default=8,
                     help="pipelined host-buffer steps (the first input copy and the last output copy are not overlapped)")
@@ -400,6 +401,45 @@ def gpu_arm(args, rank, world):
                   "note": "msa_sparse_prefill_varlen: index branch, inversion, attention and combine in one call"}
         del vt, v_out, v_lse, v_bi, v_ws
 
+    # main-branch backward on the same workload, selections held fixed: gradients of sum(dout * out) in
+    # q, k, v from the forward's out and lse of the timed steps
+    backward = None
+    if not args.no_backward:
+        bdout = to_dev(synth.normal_bf16((N, H_q, d_h), cfg.seed, "dout"))
+        bdq, bdk, bdv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
+        b_ws = torch.empty(msa.api.lib.msa_sparse_backward_workspace_size(N, H_q, H_kv, d_h, cfg.B_k, k, 0),
+                           dtype=torch.uint8, device=dev)
+
+        def backward_step():
+            msa.msa_sparse_backward(t["q"], t["k"], t["v"], out, lse, bdout, block_idx, kv, cfg.B_k, k, dq=bdq,
+                                    dk=bdk, dv=bdv, workspace=b_ws)
+
+        for _ in range(args.warmup):
+            backward_step()
+        torch.cuda.synchronize()
+        if msa.msa_get_device_error(b_ws) != 0:
+            raise RuntimeError("device error in the backward warm-up")
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        btrace = msa.KernelTrace(16 * args.steps)
+        with btrace:
+            for st in range(args.steps):
+                flush.zero_()
+                bev[st][0].record()
+                backward_step()
+                bev[st][1].record()
+        torch.cuda.synchronize()
+        (bt_ms,) = replicas.max_over_ranks([sum(a.elapsed_time(b) for a, b in bev)], device=dev)
+        bk = {n: sum(d) / args.steps for n, d in btrace.durations().items()}
+        fl_bwd = roofline.main_branch_backward_flops(N, H_q, d_h, k, cfg.B_k)
+        ach = fl_bwd / (bk["bwd_attn"] / 1000.0) / 1e12
+        backward = {"value": replicas.aggregate_rate(N * args.steps, world, bt_ms / 1000.0), "unit": UNIT,
+                    "ms_per_step": bt_ms / args.steps, "kernels_ms": bk,
+                    "roofline": {"kernel": "bwd_attn", "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
+                                 "peak": peaks["bf16_tflops"], "frac": ach / peaks["bf16_tflops"],
+                                 "algorithmic": fl_bwd},
+                    "note": "msa_sparse_backward (dq, dk, dv; selections fixed), first path on mma.sync"}
+        del bdout, bdq, bdk, bdv, b_ws
+
     # end-to-end through the public API with host buffers (pinned), copies inside the timed region:
     # every step copies its inputs in and its output back; device inputs and outputs are double
     # buffered so step s+1's inputs stream in and step s-1's output streams out while step s computes
@@ -501,6 +541,7 @@ def gpu_arm(args, rank, world):
                         "ms_per_step": dec_total / args.steps} if dcfg else None),
             "decode_graph": decode_graph,
             "roofline": roof, "kernels": kstats, "cpu_baseline": cpu_base, "e2e": e2e, "varlen": varlen,
+            "backward": backward,
             "gpu_launches": int(launches), "clocks": clocks.summary(), "wall_s_timed": wall}
     print(json.dumps(line), flush=True)
 

@@ -1,4 +1,4 @@
-"""B200 (sm_100a) MiniMax Sparse Attention forward path.
+"""B200 (sm_100a) MiniMax Sparse Attention forward path and main-branch backward.
 
 The binding (``block_sparse_long_idx_b200.api``) loads libmsa_b200.so on first use of any of its
 names, so that the seeded input generators (``block_sparse_long_idx_b200.synth``) import without
@@ -8,7 +8,7 @@ _API_NAMES = {
     "lib", "LIB_PATH", "MsaError", "KV2Q", "msa_kv2q_layout", "status_string", "msa_get_device_error",
     "msa_index_topk", "msa_kv2q_layout_get", "msa_build_kv2q", "msa_sparse_prefill_workspace_size",
     "msa_sparse_prefill", "msa_sparse_decode", "SIGNATURES", "KernelTrace", "msa_launch_count", "KERNEL_NAMES",
-    "msa_selftest_wait_timeout", "msa_sparse_prefill_varlen",
+    "msa_selftest_wait_timeout", "msa_sparse_prefill_varlen", "msa_sparse_backward",
 }
 
 

@@ -58,6 +58,9 @@ SIGNATURES = [
     ("msa_sparse_prefill_varlen_workspace_size", _sz, [_vp, _vp, _int, _int, _int, _int, _int, _int, _i64]),
     ("msa_sparse_prefill_varlen", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int,
                                          _vp, _vp, _vp, _vp, _sz, _vp]),
+    ("msa_sparse_backward_workspace_size", _sz, [_i64, _int, _int, _int, _int, _int, _int]),
+    ("msa_sparse_backward", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _int, _int, _vp, _LP, _vp,
+                                   _vp, _vp, _vp, _vp, _sz, _vp]),
     ("msa_selftest_workspace_size", _sz, []),
     ("msa_selftest_wait_timeout", _int, [_vp, _sz, _i64, _vp]),
     ("msa_trace_set", None, [_vp]),
@@ -66,7 +69,7 @@ SIGNATURES = [
 ]
 
 KERNEL_NAMES = {1: "index_topk", 2: "kv2q", 3: "attn", 4: "combine", 5: "dec_pool", 6: "dec_topk", 7: "dec_attn",
-                8: "dec_combine"}
+                8: "dec_combine", 9: "bwd_prep", 10: "bwd_attn", 11: "bwd_convert"}
 
 
 class msa_trace(ctypes.Structure):
@@ -289,6 +292,36 @@ def msa_sparse_prefill(q, k_, v, block_idx, kv2q: KV2Q | None = None, B_k: int =
         _ptr(kv2q.buf) if kv2q is not None else None, out.data_ptr(), _ptr(lse), workspace.data_ptr(),
         workspace.numel(), _stream(stream)))
     return out, lse
+
+
+def msa_sparse_backward(q, k_, v, out, lse, dout, block_idx=None, kv2q: KV2Q | None = None, B_k: int = 128,
+                        k: int | None = None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Main-branch backward with the selections held fixed: gradients of sum(dout * out) in q, k, v.
+
+    out, lse: the forward's results for the same q, k, v and selections. Returns (dq, dk, dv) bf16."""
+    for t, n in ((q, "q"), (k_, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _bf16(t, n)
+    if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse: expected a contiguous float32 CUDA tensor")
+    N, H_q, d_h = q.shape
+    H_kv = k_.shape[1]
+    if k is None:
+        if block_idx is None:
+            raise ValueError("msa_sparse_backward: k is needed when block_idx is not given")
+        k = block_idx.shape[2]
+    if kv2q is None and block_idx is None:
+        raise ValueError("msa_sparse_backward: give block_idx or a built kv2q")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k_) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = _workspace(lib.msa_sparse_backward_workspace_size(N, H_q, H_kv, d_h, B_k, k, kv2q is None), q.device,
+                    workspace)
+    lp = ctypes.byref(kv2q.layout) if kv2q is not None else None
+    _check("msa_sparse_backward", lib.msa_sparse_backward(
+        q.data_ptr(), k_.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(), N, H_q, H_kv, d_h,
+        B_k, k, _ptr(block_idx), lp, _ptr(kv2q.buf) if kv2q is not None else None, dq.data_ptr(), dk.data_ptr(),
+        dv.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 def msa_sparse_decode(q, q_idx, k_cache, v_cache, k_idx_cache, lens, B_k: int = 128, k: int = 16, out=None, lse=None,

@@ -17,6 +17,7 @@
 #include <math_constants.h>
 
 #include "common.cuh"
+#include "mma_sync.cuh"
 #include "sm100.cuh"
 #include "topk.cuh"
 
@@ -204,27 +205,6 @@ struct DecCfg {
     static_assert(4 * 16 * DH * 4 <= 128 * LD * 2, "output scratch fits in the K tile");
 };
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, const void* p)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-                 : "=r"(r0), "=r"(r1)
-                 : "r"(smem_u32(p)));
-}
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-
 template <int DH>
 __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
 {
@@ -270,7 +250,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
         else
             *reinterpret_cast<uint4*>(sQ + j * LD + u * 8) = make_uint4(0, 0, 0, 0);
     }
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+    cp_async_wait_all();
     __syncthreads();
 
     // S = Q K^T for keys 32*warp .. +31 (4 n-tiles of 8)

@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <vector>
 
+#include "backward.cuh"
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -439,6 +440,102 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
     }
     return run_passes((const uint8_t*)kv, L, N, H_q, H_kv, d_h, k, qmap, kmap, vmap, wins_per_pass, rows_pass, o_part,
                       lse_part, out, lse, workspace, s, nullptr, nullptr);
+}
+
+// ------------------------------------------------------------------------------------ backward
+size_t msa_sparse_backward_workspace_size(int64_t N, int H_q, int H_kv, int d_h, int B_k, int k, int internal_kv2q)
+{
+    msa_kv2q_layout L;
+    if (msa_kv2q_layout_get(N, H_kv, B_k, k, 0, 0, &L) != MSA_OK || H_q < 1 || d_h < 1) return 0;
+    size_t sz = kErrBytes; // error word and work counter
+    if (internal_kv2q) sz += align_up(L.total_bytes, 256) + align_up(kv2q_internal_tmp(L), 256);
+    sz += align_up((size_t)N * H_q * 4, 256);            // D = rowsum(dout * out)
+    sz += align_up((size_t)N * H_q * d_h * 4, 256);      // dq accumulator
+    sz += 2 * align_up((size_t)N * H_kv * d_h * 4, 256); // dk, dv accumulators
+    return sz;
+}
+
+msa_status msa_sparse_backward(const msa_bf16* q, const msa_bf16* kk, const msa_bf16* v, const msa_bf16* out,
+                               const float* lse, const msa_bf16* dout, int64_t N, int H_q, int H_kv, int d_h, int B_k,
+                               int k, const int32_t* block_idx, const msa_kv2q_layout* layout, const void* kv2q,
+                               msa_bf16* dq, msa_bf16* dk, msa_bf16* dv, void* workspace, size_t workspace_bytes,
+                               msa_stream_t stream)
+{
+    if (!q || !kk || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace || N < 1 || H_q < 1 || H_kv < 1 ||
+        d_h < 1 || k < 1)
+        return MSA_ERR_INVALID_ARG;
+    if ((layout == nullptr) != (kv2q == nullptr) || (!layout && !block_idx)) return MSA_ERR_INVALID_ARG;
+    if (H_q % H_kv != 0) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(kk, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 256))
+        return MSA_ERR_INVALID_ARG;
+    const int G = H_q / H_kv;
+    if (B_k != kBk || k > kMaxK || !(d_h == 64 || d_h == 128) || !pow2(G) || G > 16 || N > kMaxN)
+        return MSA_ERR_UNSUPPORTED;
+    if (layout && (!layout_ok(layout) || layout->N != N || layout->H_kv != H_kv || layout->k != k))
+        return MSA_ERR_INVALID_ARG;
+    if (injected("msa_sparse_backward")) return MSA_ERR_CUDA;
+
+    msa_kv2q_layout Lint;
+    const msa_kv2q_layout* L = layout;
+    uint8_t* ws = (uint8_t*)workspace;
+    size_t used = kErrBytes;
+    const uint8_t* kv = (const uint8_t*)kv2q;
+    void* kvbuf = nullptr;
+    void* kvtmp = nullptr;
+    if (!L) {
+        msa_kv2q_layout_get(N, H_kv, B_k, k, 0, 0, &Lint);
+        L = &Lint;
+        kvbuf = ws + used;
+        kvtmp = ws + used + align_up(L->total_bytes, 256);
+        used += align_up(L->total_bytes, 256) + align_up(kv2q_internal_tmp(*L), 256);
+        kv = (const uint8_t*)kvbuf;
+    }
+    float* D = (float*)(ws + used);
+    used += align_up((size_t)N * H_q * 4, 256);
+    uint8_t* acc0 = ws + used;
+    float* dq_acc = (float*)(ws + used);
+    used += align_up((size_t)N * H_q * d_h * 4, 256);
+    float* dk_acc = (float*)(ws + used);
+    used += align_up((size_t)N * H_kv * d_h * 4, 256);
+    float* dv_acc = (float*)(ws + used);
+    used += align_up((size_t)N * H_kv * d_h * 4, 256);
+    if (workspace_bytes < used) return MSA_ERR_WORKSPACE;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    if (kvbuf) {
+        msa_status st = build_kv2q_impl(block_idx, L, kvbuf, (int*)workspace, kvtmp, s);
+        if (st != MSA_OK) return st;
+    }
+    if (msa_status st1 = cuda_status(cudaMemsetAsync(acc0, 0, (size_t)(ws + used - acc0), s), "clearing the accumulators"))
+        return st1;
+    BwdArgs a;
+    a.N = N;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.d_h = d_h;
+    a.k = k;
+    a.q = q;
+    a.kk = kk;
+    a.v = v;
+    a.out = out;
+    a.lse = lse;
+    a.dout = dout;
+    a.entries = (const int32_t*)(kv + L->entries);
+    a.items = (const msa_work_item*)(kv + L->items);
+    a.window_items = (const int32_t*)(kv + L->window_items);
+    a.n_windows = L->n_windows;
+    a.D = D;
+    a.dq_acc = dq_acc;
+    a.dk_acc = dk_acc;
+    a.dv_acc = dv_acc;
+    a.item_counter = (int*)workspace + 4; // inside the error-word region, cleared above
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.err = (int*)workspace;
+    return cuda_status(launch_backward(a, s), "backward launch");
 }
 
 // ------------------------------------------------------------------------------------ varlen prefill

@@ -19,6 +19,13 @@ def main_branch_flops(N: int, H_q: int, d_h: int, k: int, B_k: int) -> float:
     return 4.0 * H_q * d_h * N * k * B_k
 
 
+def main_branch_backward_flops(N: int, H_q: int, d_h: int, k: int, B_k: int) -> float:
+    """Backward of the main branch with the selections fixed: per (row, head, selected block) five
+    B_k x d_h products (S recomputed, dP = dO V^T, dV += P^T dO, dK += dS^T Q, dQ += dS K), 2.5x the
+    forward's two."""
+    return 10.0 * H_q * d_h * N * k * B_k
+
+
 def index_branch_flops(N: int, H_kv: int, d_idx: int) -> float:
     return 2.0 * H_kv * d_idx * N * N / 2.0
 

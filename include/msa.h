@@ -208,6 +208,42 @@ MSA_API msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* k, cons
                               msa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Main-branch backward: gradients in q, k, v with the selections held fixed     [EXPL 03, 05]
+ *
+ * The Top-k selection is not differentiable, so the loss reaches q, k and v only through the
+ * exact attention of msa_sparse_prefill over each row's token set T. With p_j the attention
+ * weights of (i, h) (recomputed from q, k and the forward's lse), D = dout[i,h] . out[i,h] and
+ * ds_j = p_j (dout[i,h] . v[j,r] - D):
+ *   dq[i, h] = sum_{j in T} ds_j k[j, r] / sqrt(d_h)
+ *   dk[j, r] = sum over (i, h in group r) with j in T(i, r) of ds_j q[i, h] / sqrt(d_h)
+ *   dv[j, r] = sum over the same (i, h) of p_j dout[i, h]
+ * KV-outer over the inversion's work items: each item stages its K/V block once, walks its rows
+ * in 16-row tiles and keeps the block's dK and dV in registers; dq and the item's dk, dv are added
+ * to fp32 accumulators in the workspace and rounded to bf16 at the end.
+ *
+ *   q, out, dout : [N, H_q, d_h] bf16 (out: the forward's output, dout: upstream gradient)
+ *   k, v     : [N, H_kv, d_h] bf16;  lse : [N, H_q] fp32 (the forward's lse, required)
+ *   block_idx: [H_kv, N, k] int32 (the forward's selections); may be NULL when layout/kv2q are given
+ *   layout, kv2q : the forward's inversion, or both NULL to build it inside the workspace
+ *   dq : [N, H_q, d_h] bf16 out;  dk, dv : [N, H_kv, d_h] bf16 out
+ *   workspace: >= msa_sparse_backward_workspace_size(..., internal_kv2q) bytes, 256-byte aligned
+ *              (fp32 accumulators: 4 * N * d_h * (H_q + 2 * H_kv) bytes plus 4 * N * H_q)
+ * All tensor pointers 16-byte aligned (lse 4). Supported: B_k = 128, k <= 16, d_h in {64, 128},
+ * G = H_q / H_kv in {1, 2, 4, 8, 16}. Errors: MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED,
+ * MSA_ERR_WORKSPACE, MSA_ERR_CUDA; entries outside [0, N) are skipped and recorded in the device
+ * error word (MSA_ERR_DEVICE_CHECK). msa_sparse_backward_workspace_size returns 0 for arguments the
+ * call would reject.
+ * ------------------------------------------------------------------------------------------ */
+MSA_API size_t msa_sparse_backward_workspace_size(int64_t N, int H_q, int H_kv, int d_h, int B_k, int k,
+                                                  int internal_kv2q);
+
+MSA_API msa_status msa_sparse_backward(const msa_bf16* q, const msa_bf16* k, const msa_bf16* v, const msa_bf16* out,
+                                       const float* lse, const msa_bf16* dout, int64_t N, int H_q, int H_kv, int d_h,
+                                       int B_k, int kk, const int32_t* block_idx, const msa_kv2q_layout* layout,
+                                       const void* kv2q, msa_bf16* dq, msa_bf16* dk, msa_bf16* dv, void* workspace,
+                                       size_t workspace_bytes, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Packed-batch (varlen) prefill: the whole forward for B independent sequences  [EXPL 05, ABS]
  *
  * Sequence s has query rows cu_seqlens[s] .. cu_seqlens[s+1]-1 of the packed query tensors and key
@@ -290,7 +326,10 @@ typedef enum {
     MSA_KERNEL_DEC_POOL = 5,   /* decode index scores + max-pool                                */
     MSA_KERNEL_DEC_TOPK = 6,   /* decode Top-k warp merge                                       */
     MSA_KERNEL_DEC_ATTN = 7,   /* decode split attention                                        */
-    MSA_KERNEL_DEC_COMBINE = 8 /* decode LSE combine                                            */
+    MSA_KERNEL_DEC_COMBINE = 8, /* decode LSE combine                                           */
+    MSA_KERNEL_BWD_PREP = 9,    /* backward: rowsum(dout * out)                                 */
+    MSA_KERNEL_BWD_ATTN = 10,   /* backward: KV-outer gradients                                 */
+    MSA_KERNEL_BWD_CONVERT = 11 /* backward: fp32 accumulators to bf16                          */
 } msa_kernel_id;
 
 typedef struct {

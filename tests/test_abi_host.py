@@ -199,3 +199,32 @@ def test_varlen_workspace_sizes_follow_the_batch(msa):
     assert size([0, 1000, 3000], [0, 1256, 3256]) >= base      # cached prefixes (256 each) add key blocks
     single = lib.msa_sparse_prefill_workspace_size(3000, 16, 2, 128, 128, 8, 0, 1)
     assert size([0, 3000]) >= single
+
+
+def test_backward_validation_and_sizes(msa):
+    f = msa.lib.msa_sparse_backward
+    sz = msa.lib.msa_sparse_backward_workspace_size
+    N, H_q, H_kv, d_h, k = 1024, 8, 2, 64, 4
+    need = sz(N, H_q, H_kv, d_h, 128, k, 0)
+    assert need >= 4 * N * d_h * (H_q + 2 * H_kv) + 4 * N * H_q
+    assert sz(N, H_q, H_kv, d_h, 128, k, 1) > need                    # room for an internal inversion
+    assert sz(N, H_q, H_kv, d_h, 64, k, 0) == 0                       # rejected shape
+    ok = [P, P, P, P, P2, P, N, H_q, H_kv, d_h, 128, k, P, None, None, P, P, P, WS, 1 << 40, None]
+
+    def call(**kw):
+        a = list(ok)
+        names = ["q", "k", "v", "out", "lse", "dout", "N", "H_q", "H_kv", "d_h", "B_k", "kk", "block_idx", "layout",
+                 "kv2q", "dq", "dk", "dv", "ws", "ws_bytes", "stream"]
+        for n, x in kw.items():
+            a[names.index(n)] = x
+        return f(*a)
+
+    assert call(lse=None) == INVALID                  # the forward's lse is required
+    assert call(dout=None) == INVALID
+    assert call(block_idx=None) == INVALID            # neither selections nor an inversion
+    assert call(dq=P + 8) == INVALID                  # misaligned output
+    assert call(H_kv=3) == INVALID                    # H_q % H_kv
+    assert call(H_q=64, H_kv=2) == UNSUPPORTED        # G = 32
+    assert call(d_h=96) == UNSUPPORTED
+    assert call(kk=17) == UNSUPPORTED
+    assert call(ws_bytes=need - 1) == WORKSPACE
