@@ -407,29 +407,35 @@ def gpu_arm(args, rank, world):
     if not args.no_backward:
         bdout = to_dev(synth.normal_bf16((N, H_q, d_h), cfg.seed, "dout"))
         bdq, bdk, bdv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
-        b_ws = torch.empty(msa.api.lib.msa_sparse_backward_workspace_size(N, H_q, H_kv, d_h, cfg.B_k, k, 0),
+        b_ws = torch.empty(msa.api.lib.msa_sparse_backward_workspace_size(N, H_q, H_kv, d_h, cfg.B_k, k, d_idx, 0),
                            dtype=torch.uint8, device=dev)
 
-        def backward_step():
+        def backward_step(with_kl):
+            kw = dict(q_idx=t["q_idx"], k_idx=t["k_idx"], kl_weight=1.0 / (N * H_kv)) if with_kl else {}
             msa.msa_sparse_backward(t["q"], t["k"], t["v"], out, lse, bdout, block_idx, kv, cfg.B_k, k, dq=bdq,
-                                    dk=bdk, dv=bdv, workspace=b_ws)
+                                    dk=bdk, dv=bdv, workspace=b_ws, **kw)
 
-        for _ in range(args.warmup):
-            backward_step()
-        torch.cuda.synchronize()
-        if msa.msa_get_device_error(b_ws) != 0:
-            raise RuntimeError("device error in the backward warm-up")
-        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        btrace = msa.KernelTrace(16 * args.steps)
-        with btrace:
-            for st in range(args.steps):
-                flush.zero_()
-                bev[st][0].record()
-                backward_step()
-                bev[st][1].record()
-        torch.cuda.synchronize()
-        (bt_ms,) = replicas.max_over_ranks([sum(a.elapsed_time(b) for a, b in bev)], device=dev)
-        bk = {n: sum(d) / args.steps for n, d in btrace.durations().items()}
+        def timed_backward(with_kl):
+            for _ in range(args.warmup):
+                backward_step(with_kl)
+            torch.cuda.synchronize()
+            if msa.msa_get_device_error(b_ws) != 0:
+                raise RuntimeError("device error in the backward warm-up")
+            bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            btrace = msa.KernelTrace(16 * args.steps)
+            with btrace:
+                for st in range(args.steps):
+                    flush.zero_()
+                    bev[st][0].record()
+                    backward_step(with_kl)
+                    bev[st][1].record()
+            torch.cuda.synchronize()
+            (ms,) = replicas.max_over_ranks([sum(a.elapsed_time(b) for a, b in bev)], device=dev)
+            return ms, {n: sum(d) / args.steps for n, d in btrace.durations().items()}
+
+        bt_ms, bk = timed_backward(False)
+        kl_ms, kl_k = timed_backward(True)
         fl_bwd = roofline.main_branch_backward_flops(N, H_q, d_h, k, cfg.B_k)
         ach = fl_bwd / (bk["bwd_attn"] / 1000.0) / 1e12
         backward = {"value": replicas.aggregate_rate(N * args.steps, world, bt_ms / 1000.0), "unit": UNIT,
@@ -437,6 +443,9 @@ def gpu_arm(args, rank, world):
                     "roofline": {"kernel": "bwd_attn", "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
                                  "peak": peaks["bf16_tflops"], "frac": ach / peaks["bf16_tflops"],
                                  "algorithmic": fl_bwd},
+                    "with_kl": {"ms_per_step": kl_ms / args.steps, "kernels_ms": kl_k,
+                                "note": "the same call also computing the index branch's KL alignment "
+                                        "(per-row KL, dq_idx, dk_idx) in the same pass"},
                     "note": "msa_sparse_backward (dq, dk, dv; selections fixed), first path on mma.sync"}
         del bdout, bdq, bdk, bdv, b_ws
 

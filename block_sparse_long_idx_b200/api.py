@@ -58,9 +58,9 @@ SIGNATURES = [
     ("msa_sparse_prefill_varlen_workspace_size", _sz, [_vp, _vp, _int, _int, _int, _int, _int, _int, _i64]),
     ("msa_sparse_prefill_varlen", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _int,
                                          _vp, _vp, _vp, _vp, _sz, _vp]),
-    ("msa_sparse_backward_workspace_size", _sz, [_i64, _int, _int, _int, _int, _int, _int]),
+    ("msa_sparse_backward_workspace_size", _sz, [_i64, _int, _int, _int, _int, _int, _int, _int]),
     ("msa_sparse_backward", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _int, _int, _vp, _LP, _vp,
-                                   _vp, _vp, _vp, _vp, _sz, _vp]),
+                                   _vp, _vp, _vp, _vp, _vp, _int, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
     ("msa_selftest_workspace_size", _sz, []),
     ("msa_selftest_wait_timeout", _int, [_vp, _sz, _i64, _vp]),
     ("msa_trace_set", None, [_vp]),
@@ -295,10 +295,13 @@ def msa_sparse_prefill(q, k_, v, block_idx, kv2q: KV2Q | None = None, B_k: int =
 
 
 def msa_sparse_backward(q, k_, v, out, lse, dout, block_idx=None, kv2q: KV2Q | None = None, B_k: int = 128,
-                        k: int | None = None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+                        k: int | None = None, dq=None, dk=None, dv=None, q_idx=None, k_idx=None,
+                        kl_weight: float = 1.0, want_kl: bool = True, workspace=None, stream=None):
     """Main-branch backward with the selections held fixed: gradients of sum(dout * out) in q, k, v.
 
-    out, lse: the forward's results for the same q, k, v and selections. Returns (dq, dk, dv) bf16."""
+    out, lse: the forward's results for the same q, k, v and selections. Returns (dq, dk, dv) bf16.
+    With q_idx, k_idx (the index branch's inputs; needs block_idx) the same pass also returns the
+    KL alignment's gradients and per-(row, group) KL: (dq, dk, dv, dq_idx, dk_idx, kl)."""
     for t, n in ((q, "q"), (k_, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _bf16(t, n)
     if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous():
@@ -314,13 +317,27 @@ def msa_sparse_backward(q, k_, v, out, lse, dout, block_idx=None, kv2q: KV2Q | N
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k_) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    ws = _workspace(lib.msa_sparse_backward_workspace_size(N, H_q, H_kv, d_h, B_k, k, kv2q is None), q.device,
-                    workspace)
+    with_kl = q_idx is not None
+    d_idx = 0
+    dq_idx = dk_idx = kl = None
+    if with_kl:
+        _bf16(q_idx, "q_idx")
+        _bf16(k_idx, "k_idx")
+        if block_idx is None:
+            raise ValueError("msa_sparse_backward: the KL part needs block_idx")
+        d_idx = q_idx.shape[2]
+        dq_idx, dk_idx = torch.empty_like(q_idx), torch.empty_like(k_idx)
+        kl = torch.empty((N, H_kv), dtype=torch.float32, device=q.device) if want_kl else None
+    ws = _workspace(lib.msa_sparse_backward_workspace_size(N, H_q, H_kv, d_h, B_k, k, d_idx, kv2q is None),
+                    q.device, workspace)
     lp = ctypes.byref(kv2q.layout) if kv2q is not None else None
     _check("msa_sparse_backward", lib.msa_sparse_backward(
         q.data_ptr(), k_.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(), N, H_q, H_kv, d_h,
         B_k, k, _ptr(block_idx), lp, _ptr(kv2q.buf) if kv2q is not None else None, dq.data_ptr(), dk.data_ptr(),
-        dv.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)))
+        dv.data_ptr(), _ptr(q_idx), _ptr(k_idx), d_idx, float(kl_weight), _ptr(dq_idx), _ptr(dk_idx), _ptr(kl),
+        ws.data_ptr(), ws.numel(), _stream(stream)))
+    if with_kl:
+        return dq, dk, dv, dq_idx, dk_idx, kl
     return dq, dk, dv
 
 

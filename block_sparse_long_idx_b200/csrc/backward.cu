@@ -19,6 +19,15 @@
 // d_h/8-column slice each, and add it to the fp32 dq accumulator. At the end of the item dK and
 // dV are added to their fp32 accumulators (a hot block's rows are split over several items).
 // A last kernel rounds the three accumulators to bf16.
+//
+// Index-branch KL alignment (explainer section 03, "KL Loss"), optional and fused into the same
+// pass: for row i and group r over T(i, r) the student is the softmax of the unscaled index scores
+// s_j = q_idx[i,r] . k_idx[j,r], the teacher P_j the average of the group's G attention weights,
+// and KL(i, r) = sum_j P_j (log P_j - log P_idx_j); the teacher is stop-gradient, so
+//   dq_idx[i,r] += w sum_j (P_idx_j - P_j) k_idx[j,r],   dk_idx[j,r] += w (P_idx_j - P_j) q_idx[i,r].
+// A pre-pass gives each (i, r) the log-sum-exp of its index scores over T; in the KV-outer pass the
+// teacher of a position is the mean of its G rows of the P^T tile the gradient already computes,
+// and the block's k_idx rows and dk_idx accumulators stay in shared memory for the whole item.
 #include <math_constants.h>
 
 #include "backward.cuh"
@@ -33,11 +42,18 @@ constexpr int kBwdWarps = 8; // 8 x 16 keys = one 128-key block
 constexpr int kTileRows = 16;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int DH>
+template <int DH, int DI = 0>
 struct BwdCfg {
     static constexpr int LD = DH + 8;   // padded row of K, V, Q, dO (elements): conflict-free fragments
     static constexpr int LDS = kBk + 8; // padded row of dS (elements)
-    static constexpr int SMEM = (2 * kBk * LD + 2 * kTileRows * LD + kTileRows * LDS) * 2 + 3 * kTileRows * 4;
+    static constexpr int BASE = (2 * kBk * LD + 2 * kTileRows * LD + kTileRows * LDS) * 2 + 3 * kTileRows * 4;
+    // KL part (fp32): k_idx block and its dk_idx accumulators [128][DI+1], P^T [16][129], the
+    // student-minus-teacher weights [16][128], the tile's q_idx rows [16][DI] and their lse [16]
+    static constexpr int LDI = DI + 1;
+    static constexpr int LDP = kBk + 1;
+    static constexpr int KL = DI ? (2 * kBk * LDI + kTileRows * LDP + kTileRows * kBk + kTileRows * DI + kTileRows) * 4 : 0;
+    static constexpr int SMEM = BASE + KL;
+    static_assert(BASE % 16 == 0, "KL region alignment");
 };
 
 __device__ __forceinline__ uint32_t ld32(const uint16_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
@@ -70,10 +86,70 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdArgs a)
     if (lane == 0) a.D[w] = acc;
 }
 
-template <int DH, int G>
+// log-sum-exp of the unscaled index scores of (i, r) over T(i, r), one warp per (i, r); each lane
+// scores whole keys (lane + 32u of every selected block) and keeps an online (max, sum)
+template <int DI>
+__global__ void __launch_bounds__(256) kl_lse_kernel(BwdArgs a)
+{
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; // (i, r) = (w / H_kv, w % H_kv)
+    const int lane = threadIdx.x & 31;
+    if (w >= a.N * a.H_kv) return;
+    const int64_t i = w / a.H_kv;
+    const int r = (int)(w % a.H_kv);
+    float q[DI];
+    const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q_idx + w * DI);
+#pragma unroll
+    for (int d = 0; d < DI / 2; ++d) {
+        const uint32_t u = qp[d];
+        q[2 * d] = bf_lo(u);
+        q[2 * d + 1] = bf_hi(u);
+    }
+    float m = -CUDART_INF_F, l = 0.f;
+    const int32_t* sel = a.block_idx + ((int64_t)r * a.N + i) * a.k;
+    for (int s = 0; s < a.k; ++s) {
+        const int32_t b = sel[s];
+        if (b < 0 || (int64_t)b * kBk > i) continue;
+#pragma unroll
+        for (int u = 0; u < kBk / 32; ++u) {
+            const int64_t j = (int64_t)b * kBk + lane + 32 * u;
+            if (j > i) continue;
+            const uint4* kp = reinterpret_cast<const uint4*>(a.k_idx + (j * a.H_kv + r) * DI);
+            float sdot = 0.f;
+#pragma unroll
+            for (int c = 0; c < DI / 8; ++c) {
+                const uint4 x = kp[c];
+                sdot = fmaf(q[8 * c + 0], bf_lo(x.x), sdot);
+                sdot = fmaf(q[8 * c + 1], bf_hi(x.x), sdot);
+                sdot = fmaf(q[8 * c + 2], bf_lo(x.y), sdot);
+                sdot = fmaf(q[8 * c + 3], bf_hi(x.y), sdot);
+                sdot = fmaf(q[8 * c + 4], bf_lo(x.z), sdot);
+                sdot = fmaf(q[8 * c + 5], bf_hi(x.z), sdot);
+                sdot = fmaf(q[8 * c + 6], bf_lo(x.w), sdot);
+                sdot = fmaf(q[8 * c + 7], bf_hi(x.w), sdot);
+            }
+            if (sdot > m) {
+                l = l * expf(m - sdot) + 1.f;
+                m = sdot;
+            } else {
+                l += expf(sdot - m);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+        const float M = fmaxf(m, m2);
+        l = (m == -CUDART_INF_F ? 0.f : l * expf(m - M)) + (m2 == -CUDART_INF_F ? 0.f : l2 * expf(m2 - M));
+        m = M;
+    }
+    if (lane == 0) a.lse_idx[w] = m + logf(l);
+}
+
+template <int DH, int G, int DI>
 __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
 {
-    using C = BwdCfg<DH>;
+    using C = BwdCfg<DH, DI>;
     constexpr int LD = C::LD, LDS = C::LDS;
     constexpr int PPT = kTileRows / G; // positions per tile
     constexpr int CPR = DH / 8;        // 16-byte chunks per row
@@ -87,6 +163,14 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
     float* sLse = reinterpret_cast<float*>(sdS + kTileRows * LDS); // lse * log2e (+inf: no row)
     float* sD = sLse + kTileRows;
     int* sPos = reinterpret_cast<int*>(sD + kTileRows); // query position of each tile row (-1: none)
+    // KL part (unused when DI == 0)
+    constexpr int LDI = C::LDI, LDP = C::LDP;
+    float* sKI = reinterpret_cast<float*>(smem_raw + C::BASE); // [128][LDI] k_idx of the block
+    float* sDKI = sKI + kBk * LDI;                             // [128][LDI] dk_idx of the block
+    float* sP = sDKI + kBk * LDI;                              // [16][LDP] P^T of the tile (row-major)
+    float* sG = sP + kTileRows * LDP;                          // [PPT][128] w (P_idx - P) per position, key
+    float* sQI = sG + kTileRows * kBk;                         // [PPT][DI] q_idx of the tile's positions
+    float* sLI = sQI + kTileRows * (DI > 0 ? DI : 1);           // [PPT] lse of the index scores
     __shared__ int s_item;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -122,6 +206,18 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
             } else {
                 *reinterpret_cast<uint4*>(sK + jj * LD + u * 8) = make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4*>(sV + jj * LD + u * 8) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        if constexpr (DI > 0) {
+            for (int c = tid; c < kBk * DI; c += kBwdWarps * 32) {
+                const int jj = c / DI, d = c % DI;
+                float x = 0.f;
+                if (tok0 + jj < a.N) {
+                    const uint16_t u = a.k_idx[((tok0 + jj) * a.H_kv + r) * DI + d];
+                    x = __uint_as_float((uint32_t)u << 16);
+                }
+                sKI[jj * LDI + d] = x;
+                sDKI[jj * LDI + d] = 0.f;
             }
         }
         float dk[DH / 8][4], dv[DH / 8][4];
@@ -161,6 +257,18 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
                 } else {
                     *reinterpret_cast<uint4*>(sQ + row * LD + u * 8) = make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4*>(sdO + row * LD + u * 8) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            if constexpr (DI > 0) {
+                for (int c = tid; c < PPT * DI; c += kBwdWarps * 32) {
+                    const int pl = c / DI, d = c % DI;
+                    const int pos = sPos[pl * G];
+                    sQI[c] = pos >= 0 ? __uint_as_float((uint32_t)a.q_idx[((int64_t)pos * a.H_kv + r) * DI + d] << 16)
+                                      : 0.f;
+                }
+                if (tid < PPT) {
+                    const int pos = sPos[tid * G];
+                    sLI[tid] = pos >= 0 ? a.lse_idx[(int64_t)pos * a.H_kv + r] : 0.f;
                 }
             }
             cp_async_wait_all();
@@ -221,6 +329,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
                     const int key = kw0 + g + ((q & 2) ? 8 : 0);
                     const int row = n * 8 + 2 * t + (q & 1);
                     sdS[row * LDS + key] = (uint16_t)(pack_bf16x2(dpt[n][q], 0.f) & 0xffffu);
+                    if constexpr (DI > 0) sP[row * LDP + key] = st[n][q];
                 }
             __syncthreads();
             // dQ of the tile, columns warp*DH/8 .. +DH/8: dS (16 x 128 keys) K (128 keys x DH)
@@ -251,9 +360,56 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
                     if (pos >= 0)
                         atomicAdd(a.dq_acc + ((int64_t)pos * a.H_q + r * G + row % G) * DH + col, scale * dq[n][q]);
                 }
+            if constexpr (DI > 0) {
+                // per (position, key): teacher = mean of the position's G rows of P^T, student weight
+                // from the index score; thread = (key j, half of the d_idx dimensions)
+                const int j = tid & (kBk - 1), half = tid >> 7;
+                const int64_t key = tok0 + j;
+                for (int pl = 0; pl < PPT; ++pl) {
+                    const int pos = sPos[pl * G];
+                    const bool valid = pos >= 0 && key <= pos;
+                    float T = 0.f;
+#pragma unroll
+                    for (int hh = 0; hh < G; ++hh) T += sP[(pl * G + hh) * LDP + j];
+                    T *= 1.f / G;
+                    float sidx = 0.f;
+#pragma unroll 8
+                    for (int d = 0; d < DI; ++d) sidx = fmaf(sQI[pl * DI + d], sKI[j * LDI + d], sidx);
+                    const float lq = sidx - sLI[pl]; // log of the student weight
+                    const float gw = valid ? a.kl_weight * (expf(lq) - T) : 0.f;
+                    if (half == 0) sG[pl * kBk + j] = gw;
+#pragma unroll 8
+                    for (int d = half * (DI / 2); d < (half + 1) * (DI / 2); ++d)
+                        sDKI[j * LDI + d] = fmaf(gw, sQI[pl * DI + d], sDKI[j * LDI + d]);
+                    if (a.kl != nullptr && half == 0) { // warp-uniform
+                        float term = (valid && T > 0.f) ? T * (logf(T) - lq) : 0.f;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) term += __shfl_xor_sync(0xffffffffu, term, o);
+                        if (lane == 0 && pos >= 0) atomicAdd(a.kl + (int64_t)pos * a.H_kv + r, term);
+                    }
+                }
+                __syncthreads();
+                // dq_idx of each position: sum over the block's keys of w (P_idx - P) k_idx
+                for (int c = tid; c < PPT * DI; c += kBwdWarps * 32) {
+                    const int pl = c / DI, d = c % DI;
+                    const int pos = sPos[pl * G];
+                    if (pos < 0) continue;
+                    float acc = 0.f;
+#pragma unroll 8
+                    for (int jj = 0; jj < kBk; ++jj) acc = fmaf(sG[pl * kBk + jj], sKI[jj * LDI + d], acc);
+                    atomicAdd(a.dqi_acc + ((int64_t)pos * a.H_kv + r) * DI + d, acc);
+                }
+            }
             __syncthreads(); // sQ, sdO, sdS and the row tables are free for the next tile
         }
         cp_async_wait_all(); // an item without rows still has its K/V copies in flight
+        if constexpr (DI > 0) {
+            __syncthreads(); // every thread's dk_idx updates (or, without rows, the zeroing) are visible
+            for (int c = tid; c < kBk * DI; c += kBwdWarps * 32) {
+                const int jj = c / DI, d = c % DI;
+                if (tok0 + jj < a.N) atomicAdd(a.dki_acc + ((tok0 + jj) * a.H_kv + r) * DI + d, sDKI[jj * LDI + d]);
+            }
+        }
         // the warp's keys: dK and dV into the fp32 accumulators
 #pragma unroll
         for (int n = 0; n < DH / 8; ++n)
@@ -280,33 +436,43 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(const float* __restric
     }
 }
 
-template <int DH, int G>
+template <int DH, int G, int DI>
 cudaError_t launch_attn_cfg(const BwdArgs& a, cudaStream_t s, int n_sm)
 {
-    const int smem = BwdCfg<DH>::SMEM;
-    cudaError_t e = cudaFuncSetAttribute(bwd_attn_kernel<DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = BwdCfg<DH, DI>::SMEM;
+    static_assert(BwdCfg<DH, DI>::SMEM <= 227 * 1024, "shared memory budget");
+    cudaError_t e = cudaFuncSetAttribute(bwd_attn_kernel<DH, G, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_attn_kernel<DH, G>, kBwdWarps * 32, smem) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_attn_kernel<DH, G, DI>, kBwdWarps * 32, smem) !=
             cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
-    bwd_attn_kernel<DH, G><<<n_sm * per_sm, kBwdWarps * 32, smem, s>>>(a);
+    bwd_attn_kernel<DH, G, DI><<<n_sm * per_sm, kBwdWarps * 32, smem, s>>>(a);
     note_launch(1);
     return cudaGetLastError();
+}
+
+template <int DH, int DI>
+cudaError_t launch_attn_g(const BwdArgs& a, int G, cudaStream_t s, int n_sm)
+{
+    switch (G) {
+    case 1: return launch_attn_cfg<DH, 1, DI>(a, s, n_sm);
+    case 2: return launch_attn_cfg<DH, 2, DI>(a, s, n_sm);
+    case 4: return launch_attn_cfg<DH, 4, DI>(a, s, n_sm);
+    case 8: return launch_attn_cfg<DH, 8, DI>(a, s, n_sm);
+    case 16: return launch_attn_cfg<DH, 16, DI>(a, s, n_sm);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 template <int DH>
 cudaError_t launch_attn_dh(const BwdArgs& a, int G, cudaStream_t s, int n_sm)
 {
-    switch (G) {
-    case 1: return launch_attn_cfg<DH, 1>(a, s, n_sm);
-    case 2: return launch_attn_cfg<DH, 2>(a, s, n_sm);
-    case 4: return launch_attn_cfg<DH, 4>(a, s, n_sm);
-    case 8: return launch_attn_cfg<DH, 8>(a, s, n_sm);
-    case 16: return launch_attn_cfg<DH, 16>(a, s, n_sm);
-    default: return cudaErrorInvalidValue;
-    }
+    if (a.q_idx == nullptr) return launch_attn_g<DH, 0>(a, G, s, n_sm);
+    if (a.d_idx == 32) return launch_attn_g<DH, 32>(a, G, s, n_sm);
+    if (a.d_idx == 64) return launch_attn_g<DH, 64>(a, G, s, n_sm);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_convert(const float* src, uint16_t* dst, int64_t n, cudaStream_t s, int n_sm)
@@ -336,6 +502,14 @@ cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s)
     else
         bwd_prep_kernel<64><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(a);
     note_launch(1);
+    if (a.q_idx != nullptr) {
+        const int64_t wk = a.N * a.H_kv;
+        if (a.d_idx == 64)
+            kl_lse_kernel<64><<<(unsigned)((wk + 7) / 8), 256, 0, s>>>(a);
+        else
+            kl_lse_kernel<32><<<(unsigned)((wk + 7) / 8), 256, 0, s>>>(a);
+        note_launch(1);
+    }
     trace_end(s, MSA_KERNEL_BWD_PREP);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -349,6 +523,10 @@ cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s)
     e = launch_convert(a.dq_acc, a.dq, a.N * a.H_q * a.d_h, s, n_sm);
     if (e == cudaSuccess) e = launch_convert(a.dk_acc, a.dk, a.N * a.H_kv * a.d_h, s, n_sm);
     if (e == cudaSuccess) e = launch_convert(a.dv_acc, a.dv, a.N * a.H_kv * a.d_h, s, n_sm);
+    if (e == cudaSuccess && a.q_idx != nullptr) {
+        e = launch_convert(a.dqi_acc, a.dq_idx, a.N * a.H_kv * a.d_idx, s, n_sm);
+        if (e == cudaSuccess) e = launch_convert(a.dki_acc, a.dk_idx, a.N * a.H_kv * a.d_idx, s, n_sm);
+    }
     trace_end(s, MSA_KERNEL_BWD_CONVERT);
     return e;
 }

@@ -30,10 +30,23 @@ struct BwdArgs {
     uint16_t* dk;  // [N, H_kv, d_h]
     uint16_t* dv;  // [N, H_kv, d_h]
     int* err;
+    // index-branch KL alignment, fused into the same pass (q_idx == nullptr: skipped)
+    const uint16_t* q_idx = nullptr;     // [N, H_kv, d_idx] bf16
+    const uint16_t* k_idx = nullptr;     // [N, H_kv, d_idx] bf16
+    const int32_t* block_idx = nullptr;  // [H_kv, N, k] selections
+    int d_idx = 0;                       // 32 or 64
+    float kl_weight = 1.f;               // gradients of kl_weight * sum of KL(i, r)
+    float* lse_idx = nullptr;            // [N, H_kv] workspace: log-sum-exp of the index scores over T
+    float* dqi_acc = nullptr;            // [N, H_kv, d_idx] fp32 accumulators (zeroed before the launch)
+    float* dki_acc = nullptr;
+    float* kl = nullptr;                 // [N, H_kv] KL(i, r) (zeroed before the launch), or nullptr
+    uint16_t* dq_idx = nullptr;          // [N, H_kv, d_idx] bf16 results
+    uint16_t* dk_idx = nullptr;
 };
 
-// D = rowsum(dout * out); the KV-outer gradient kernel; the fp32 -> bf16 conversion of the three
-// gradients. The accumulators must be zero before the first.
+// D = rowsum(dout * out) (and, with the KL part, the index log-sum-exp over each row's token set);
+// the KV-outer gradient kernel; the fp32 -> bf16 conversion of the gradients. The accumulators
+// (and kl) must be zero before the first.
 cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s);
 
 } // namespace msa

@@ -443,23 +443,27 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
 }
 
 // ------------------------------------------------------------------------------------ backward
-size_t msa_sparse_backward_workspace_size(int64_t N, int H_q, int H_kv, int d_h, int B_k, int k, int internal_kv2q)
+size_t msa_sparse_backward_workspace_size(int64_t N, int H_q, int H_kv, int d_h, int B_k, int k, int d_idx,
+                                          int internal_kv2q)
 {
     msa_kv2q_layout L;
     if (msa_kv2q_layout_get(N, H_kv, B_k, k, 0, 0, &L) != MSA_OK || H_q < 1 || d_h < 1) return 0;
+    if (d_idx != 0 && d_idx != 32 && d_idx != 64) return 0;
     size_t sz = kErrBytes; // error word and work counter
     if (internal_kv2q) sz += align_up(L.total_bytes, 256) + align_up(kv2q_internal_tmp(L), 256);
     sz += align_up((size_t)N * H_q * 4, 256);            // D = rowsum(dout * out)
     sz += align_up((size_t)N * H_q * d_h * 4, 256);      // dq accumulator
     sz += 2 * align_up((size_t)N * H_kv * d_h * 4, 256); // dk, dv accumulators
+    if (d_idx) sz += align_up((size_t)N * H_kv * 4, 256) + 2 * align_up((size_t)N * H_kv * d_idx * 4, 256);
     return sz;
 }
 
 msa_status msa_sparse_backward(const msa_bf16* q, const msa_bf16* kk, const msa_bf16* v, const msa_bf16* out,
                                const float* lse, const msa_bf16* dout, int64_t N, int H_q, int H_kv, int d_h, int B_k,
                                int k, const int32_t* block_idx, const msa_kv2q_layout* layout, const void* kv2q,
-                               msa_bf16* dq, msa_bf16* dk, msa_bf16* dv, void* workspace, size_t workspace_bytes,
-                               msa_stream_t stream)
+                               msa_bf16* dq, msa_bf16* dk, msa_bf16* dv, const msa_bf16* q_idx, const msa_bf16* k_idx,
+                               int d_idx, float kl_weight, msa_bf16* dq_idx, msa_bf16* dk_idx, float* kl,
+                               void* workspace, size_t workspace_bytes, msa_stream_t stream)
 {
     if (!q || !kk || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace || N < 1 || H_q < 1 || H_kv < 1 ||
         d_h < 1 || k < 1)
@@ -474,6 +478,13 @@ msa_status msa_sparse_backward(const msa_bf16* q, const msa_bf16* kk, const msa_
         return MSA_ERR_UNSUPPORTED;
     if (layout && (!layout_ok(layout) || layout->N != N || layout->H_kv != H_kv || layout->k != k))
         return MSA_ERR_INVALID_ARG;
+    const bool with_kl = q_idx != nullptr;
+    if (with_kl) {
+        if (!k_idx || !dq_idx || !dk_idx || !block_idx || !aligned(q_idx, 16) || !aligned(k_idx, 16) ||
+            !aligned(dq_idx, 16) || !aligned(dk_idx, 16) || (kl && !aligned(kl, 4)))
+            return MSA_ERR_INVALID_ARG;
+        if (d_idx != 32 && d_idx != 64) return MSA_ERR_UNSUPPORTED;
+    }
     if (injected("msa_sparse_backward")) return MSA_ERR_CUDA;
 
     msa_kv2q_layout Lint;
@@ -500,6 +511,16 @@ msa_status msa_sparse_backward(const msa_bf16* q, const msa_bf16* kk, const msa_
     used += align_up((size_t)N * H_kv * d_h * 4, 256);
     float* dv_acc = (float*)(ws + used);
     used += align_up((size_t)N * H_kv * d_h * 4, 256);
+    float *dqi_acc = nullptr, *dki_acc = nullptr, *lse_idx = nullptr;
+    if (with_kl) {
+        dqi_acc = (float*)(ws + used);
+        used += align_up((size_t)N * H_kv * d_idx * 4, 256);
+        dki_acc = (float*)(ws + used);
+        used += align_up((size_t)N * H_kv * d_idx * 4, 256);
+        lse_idx = (float*)(ws + used); // written before it is read: outside the cleared range
+        used += align_up((size_t)N * H_kv * 4, 256);
+    }
+    const size_t acc_bytes = (size_t)((lse_idx ? (uint8_t*)lse_idx : ws + used) - acc0);
     if (workspace_bytes < used) return MSA_ERR_WORKSPACE;
 
     cudaStream_t s = (cudaStream_t)stream;
@@ -508,8 +529,10 @@ msa_status msa_sparse_backward(const msa_bf16* q, const msa_bf16* kk, const msa_
         msa_status st = build_kv2q_impl(block_idx, L, kvbuf, (int*)workspace, kvtmp, s);
         if (st != MSA_OK) return st;
     }
-    if (msa_status st1 = cuda_status(cudaMemsetAsync(acc0, 0, (size_t)(ws + used - acc0), s), "clearing the accumulators"))
+    if (msa_status st1 = cuda_status(cudaMemsetAsync(acc0, 0, acc_bytes, s), "clearing the accumulators"))
         return st1;
+    if (with_kl && kl)
+        if (msa_status st2 = cuda_status(cudaMemsetAsync(kl, 0, (size_t)N * H_kv * 4, s), "clearing kl")) return st2;
     BwdArgs a;
     a.N = N;
     a.H_q = H_q;
@@ -535,6 +558,19 @@ msa_status msa_sparse_backward(const msa_bf16* q, const msa_bf16* kk, const msa_
     a.dk = dk;
     a.dv = dv;
     a.err = (int*)workspace;
+    if (with_kl) {
+        a.q_idx = q_idx;
+        a.k_idx = k_idx;
+        a.block_idx = block_idx;
+        a.d_idx = d_idx;
+        a.kl_weight = kl_weight;
+        a.lse_idx = lse_idx;
+        a.dqi_acc = dqi_acc;
+        a.dki_acc = dki_acc;
+        a.kl = kl;
+        a.dq_idx = dq_idx;
+        a.dk_idx = dk_idx;
+    }
     return cuda_status(launch_backward(a, s), "backward launch");
 }
 

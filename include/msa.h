@@ -208,7 +208,7 @@ MSA_API msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* k, cons
                               msa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
- * Main-branch backward: gradients in q, k, v with the selections held fixed     [EXPL 03, 05]
+ * Backward: main-branch gradients (selections fixed) and the index-branch KL signal [EXPL 03, 05]
  *
  * The Top-k selection is not differentiable, so the loss reaches q, k and v only through the
  * exact attention of msa_sparse_prefill over each row's token set T. With p_j the attention
@@ -221,26 +221,40 @@ MSA_API msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* k, cons
  * in 16-row tiles and keeps the block's dK and dV in registers; dq and the item's dk, dv are added
  * to fp32 accumulators in the workspace and rounded to bf16 at the end.
  *
+ * Optional, in the same pass (q_idx != NULL): the index branch's KL alignment [EXPL 03 "KL Loss"].
+ * Over T(i, r) the student is P_idx = softmax(q_idx[i,r] . k_idx[j,r]) (unscaled index scores), the
+ * teacher P = the mean of the group's G attention weights above; KL(i, r) = sum_j P_j log(P_j /
+ * P_idx_j), teacher stop-gradient, so with w = kl_weight (1 / (N * H_kv) for the mean):
+ *   dq_idx[i, r] = w sum_{j in T} (P_idx_j - P_j) k_idx[j, r]
+ *   dk_idx[j, r] = w sum over rows i with j in T(i, r) of (P_idx_j - P_j) q_idx[i, r]
+ *   kl[i, r]     = KL(i, r) (unweighted), when kl != NULL
+ *
  *   q, out, dout : [N, H_q, d_h] bf16 (out: the forward's output, dout: upstream gradient)
  *   k, v     : [N, H_kv, d_h] bf16;  lse : [N, H_q] fp32 (the forward's lse, required)
  *   block_idx: [H_kv, N, k] int32 (the forward's selections); may be NULL when layout/kv2q are given
  *   layout, kv2q : the forward's inversion, or both NULL to build it inside the workspace
  *   dq : [N, H_q, d_h] bf16 out;  dk, dv : [N, H_kv, d_h] bf16 out
- *   workspace: >= msa_sparse_backward_workspace_size(..., internal_kv2q) bytes, 256-byte aligned
- *              (fp32 accumulators: 4 * N * d_h * (H_q + 2 * H_kv) bytes plus 4 * N * H_q)
+ *   q_idx, k_idx : [N, H_kv, d_idx] bf16 (the index branch's inputs), or q_idx = NULL to skip the KL
+ *              part (then k_idx, d_idx, kl_weight, dq_idx, dk_idx, kl are ignored); needs block_idx
+ *   dq_idx, dk_idx : [N, H_kv, d_idx] bf16 out;  kl : [N, H_kv] fp32 out, or NULL
+ *   workspace: >= msa_sparse_backward_workspace_size(..., d_idx or 0 without KL, internal_kv2q) bytes,
+ *              256-byte aligned (fp32 accumulators: 4 * N * d_h * (H_q + 2 * H_kv) bytes plus
+ *              4 * N * H_q, and with KL 4 * N * H_kv * (2 * d_idx + 1))
  * All tensor pointers 16-byte aligned (lse 4). Supported: B_k = 128, k <= 16, d_h in {64, 128},
- * G = H_q / H_kv in {1, 2, 4, 8, 16}. Errors: MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED,
- * MSA_ERR_WORKSPACE, MSA_ERR_CUDA; entries outside [0, N) are skipped and recorded in the device
- * error word (MSA_ERR_DEVICE_CHECK). msa_sparse_backward_workspace_size returns 0 for arguments the
- * call would reject.
+ * G = H_q / H_kv in {1, 2, 4, 8, 16}, d_idx in {32, 64} for the KL part. Errors:
+ * MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA; entries outside
+ * [0, N) are skipped and recorded in the device error word (MSA_ERR_DEVICE_CHECK).
+ * msa_sparse_backward_workspace_size returns 0 for arguments the call would reject.
  * ------------------------------------------------------------------------------------------ */
 MSA_API size_t msa_sparse_backward_workspace_size(int64_t N, int H_q, int H_kv, int d_h, int B_k, int k,
-                                                  int internal_kv2q);
+                                                  int d_idx, int internal_kv2q);
 
 MSA_API msa_status msa_sparse_backward(const msa_bf16* q, const msa_bf16* k, const msa_bf16* v, const msa_bf16* out,
                                        const float* lse, const msa_bf16* dout, int64_t N, int H_q, int H_kv, int d_h,
                                        int B_k, int kk, const int32_t* block_idx, const msa_kv2q_layout* layout,
-                                       const void* kv2q, msa_bf16* dq, msa_bf16* dk, msa_bf16* dv, void* workspace,
+                                       const void* kv2q, msa_bf16* dq, msa_bf16* dk, msa_bf16* dv,
+                                       const msa_bf16* q_idx, const msa_bf16* k_idx, int d_idx, float kl_weight,
+                                       msa_bf16* dq_idx, msa_bf16* dk_idx, float* kl, void* workspace,
                                        size_t workspace_bytes, msa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------

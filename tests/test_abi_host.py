@@ -205,16 +205,20 @@ def test_backward_validation_and_sizes(msa):
     f = msa.lib.msa_sparse_backward
     sz = msa.lib.msa_sparse_backward_workspace_size
     N, H_q, H_kv, d_h, k = 1024, 8, 2, 64, 4
-    need = sz(N, H_q, H_kv, d_h, 128, k, 0)
+    need = sz(N, H_q, H_kv, d_h, 128, k, 0, 0)
     assert need >= 4 * N * d_h * (H_q + 2 * H_kv) + 4 * N * H_q
-    assert sz(N, H_q, H_kv, d_h, 128, k, 1) > need                    # room for an internal inversion
-    assert sz(N, H_q, H_kv, d_h, 64, k, 0) == 0                       # rejected shape
-    ok = [P, P, P, P, P2, P, N, H_q, H_kv, d_h, 128, k, P, None, None, P, P, P, WS, 1 << 40, None]
+    assert sz(N, H_q, H_kv, d_h, 128, k, 0, 1) > need                 # room for an internal inversion
+    assert sz(N, H_q, H_kv, d_h, 128, k, 64, 0) >= need + 4 * N * H_kv * (2 * 64 + 1)  # KL accumulators
+    assert sz(N, H_q, H_kv, d_h, 64, k, 0, 0) == 0                    # rejected shape
+    assert sz(N, H_q, H_kv, d_h, 128, k, 48, 0) == 0                  # rejected d_idx
+    ok = [P, P, P, P, P2, P, N, H_q, H_kv, d_h, 128, k, P, None, None, P, P, P, None, None, 0, 1.0, None, None, None,
+          WS, 1 << 40, None]
+    names = ["q", "k", "v", "out", "lse", "dout", "N", "H_q", "H_kv", "d_h", "B_k", "kk", "block_idx", "layout",
+             "kv2q", "dq", "dk", "dv", "q_idx", "k_idx", "d_idx", "kl_weight", "dq_idx", "dk_idx", "kl", "ws",
+             "ws_bytes", "stream"]
 
     def call(**kw):
         a = list(ok)
-        names = ["q", "k", "v", "out", "lse", "dout", "N", "H_q", "H_kv", "d_h", "B_k", "kk", "block_idx", "layout",
-                 "kv2q", "dq", "dk", "dv", "ws", "ws_bytes", "stream"]
         for n, x in kw.items():
             a[names.index(n)] = x
         return f(*a)
@@ -228,3 +232,9 @@ def test_backward_validation_and_sizes(msa):
     assert call(d_h=96) == UNSUPPORTED
     assert call(kk=17) == UNSUPPORTED
     assert call(ws_bytes=need - 1) == WORKSPACE
+    kl = dict(q_idx=P, k_idx=P, d_idx=64, dq_idx=P, dk_idx=P, kl=P2)
+    assert call(**dict(kl, dk_idx=None)) == INVALID      # KL outputs required with q_idx
+    assert call(**dict(kl, block_idx=None)) == INVALID   # the KL part reads the selections
+    assert call(**dict(kl, k_idx=P + 2)) == INVALID      # misaligned
+    assert call(**dict(kl, d_idx=128)) == UNSUPPORTED
+    assert call(**dict(kl, ws_bytes=need)) == WORKSPACE  # no room for the KL accumulators

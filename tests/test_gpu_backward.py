@@ -1,7 +1,8 @@
-"""GPU parity, main-branch backward: dq, dk, dv of the CUDA path against the CPU oracle's gradients
+"""GPU parity, backward: dq, dk, dv of the CUDA path against the CPU oracle's gradients
 (selections held fixed), on small shapes in full and on sampled rows / blocks, plus the two sums
 that hold at any size (sum_j dv[j, r] = sum of the group's dout; sum_j dk[j, r] = 0) on the 128K
-planted workload.
+planted workload; and the index-branch KL alignment fused into the same pass (per-row KL, dq_idx,
+dk_idx against the oracle; sum_j dk_idx[j, r] = 0 at 128K).
 
 Tolerance (gradients are bf16 outputs of products whose operands P and dS are rounded to bf16,
 accumulated in fp32; each rounding is 2^-9 relative): per tensor, max |d| <= 2e-2 * max |ref| + 1e-5
@@ -100,7 +101,7 @@ def test_backward_internal_inversion_and_error_word():
     cfg = _cfg("internal", 1300, 8, 2, 64, 32, 5)
     inp = synth.prefill_inputs(cfg)
     dout = synth.normal_bf16((cfg.N, cfg.H_q, cfg.d_h), cfg.seed, "dout")
-    nbytes = msa.lib.msa_sparse_backward_workspace_size(cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, 128, cfg.k, 1)
+    nbytes = msa.lib.msa_sparse_backward_workspace_size(cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, 128, cfg.k, 0, 1)
     ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     dq, dk, dv = _forward_backward(cfg, inp, dout, use_kv=False, workspace=ws)
     assert msa.msa_get_device_error(ws) == 0
@@ -134,3 +135,74 @@ def test_backward_128k_planted_sampled():
         assert np.max(np.abs(got - want)) <= 1e-2 * np.abs(dv[:, r]).sum(axis=0).max(), r
         sk = dk[:, r].sum(axis=0)                                # softmax Jacobian rows sum to zero
         assert np.max(np.abs(sk)) <= 1e-2 * np.abs(dk[:, r]).sum(axis=0).max(), r
+
+
+def _forward_backward_kl(cfg, inp, dout, w):
+    t = {n: dev(a) for n, a in inp.items()}
+    bi = msa.msa_index_topk(t["q_idx"], t["k_idx"], 128, cfg.k)
+    kv = msa.msa_build_kv2q(bi, 128)
+    out, lse = msa.msa_sparse_prefill(t["q"], t["k"], t["v"], bi, kv)
+    res = msa.msa_sparse_backward(t["q"], t["k"], t["v"], out, lse, dev(dout), bi, kv, q_idx=t["q_idx"],
+                                  k_idx=t["k_idx"], kl_weight=w)
+    torch.cuda.synchronize()
+    dq, dk, dv, dqi, dki, kl = res
+    return (bf16_to_f64(dq), bf16_to_f64(dk), bf16_to_f64(dv), bf16_to_f64(dqi), bf16_to_f64(dki),
+            kl.cpu().numpy().astype(np.float64))
+
+
+KL_CASES = [
+    # name, N, H_q, H_kv, d_h, d_idx, k, full
+    ("kl_tiny_N2048_G4_didx32", 2048, 8, 2, 64, 32, 4, True),
+    ("kl_G16_N1500_didx64", 1500, 32, 2, 128, 64, 8, False),
+    ("kl_G1_N700", 700, 2, 2, 128, 64, 3, True),
+]
+
+
+@pytest.mark.parametrize("case", KL_CASES, ids=[c[0] for c in KL_CASES])
+def test_backward_with_kl(case):
+    """The KL alignment's per-(row, group) value and gradients in q_idx and k_idx, and the main-branch
+    gradients of the same call (the KL part must leave them as without it)."""
+    name, N, H_q, H_kv, d_h, d_idx, k, full = case
+    cfg = _cfg(name, N, H_q, H_kv, d_h, d_idx, k)
+    inp = synth.prefill_inputs(cfg)
+    dout = synth.normal_bf16((N, H_q, d_h), cfg.seed, "dout")
+    w = 0.5
+    dq, dk, dv, dqi, dki, kl = _forward_backward_kl(cfg, inp, dout, w)
+    sel = oracle.select_rows(inp["q_idx"], inp["k_idx"], np.arange(N), 128, k)
+    rows = np.arange(N) if full else synth.sample_rows(N, 128, 200, 5)
+    want_kl, want_dqi = oracle.kl_rows(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], rows, sel[rows], 128, w)
+    assert_grad_close(kl[rows], want_kl, "kl")
+    assert_grad_close(dqi[rows], want_dqi, "dq_idx")
+    want_dq = oracle.backward_dq_rows(inp["q"], dout, inp["k"], inp["v"], rows, sel[rows], 128)
+    assert_grad_close(dq[rows], want_dq, "dq")
+    nb = (N + 127) // 128
+    pairs = ([(r, b) for r in range(H_kv) for b in range(nb)] if full
+             else sorted({(0, 0), (H_kv - 1, nb - 1), (0, nb // 2), (H_kv - 1, 1)}))
+    want_dki = oracle.kl_dk_idx_blocks(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], sel, pairs, 128, w)
+    got_dki = np.stack([np.pad(dki[b * 128:(b + 1) * 128, r], ((0, 128 - len(dki[b * 128:(b + 1) * 128])), (0, 0)))
+                        for r, b in pairs])
+    assert_grad_close(got_dki, want_dki, "dk_idx")
+    want_dk, want_dv = oracle.backward_dkv_blocks(inp["q"], dout, inp["k"], inp["v"], sel, pairs, 128)
+    got_dv = np.stack([np.pad(dv[b * 128:(b + 1) * 128, r], ((0, 128 - len(dv[b * 128:(b + 1) * 128])), (0, 0)))
+                       for r, b in pairs])
+    assert_grad_close(got_dv, want_dv, "dv")
+
+
+def test_backward_kl_128k_planted_sampled():
+    """The 128K planted workload with the KL part: KL and dq_idx on sampled rows against the oracle
+    (its own selections of those rows), and sum_j dk_idx[j, r] = 0 (student and teacher both sum to
+    one over every row's token set)."""
+    cfg = synth.P128K
+    inp = synth.prefill_inputs(cfg)
+    dout = synth.normal_bf16((cfg.N, cfg.H_q, cfg.d_h), cfg.seed, "dout")
+    w = 1.0 / (cfg.N * cfg.H_kv)
+    _, _, _, dqi, dki, kl = _forward_backward_kl(cfg, inp, dout, w)
+    rows = synth.sample_rows(cfg.N, 128, 48, 13)
+    sel = oracle.select_rows(inp["q_idx"], inp["k_idx"], rows, 128, cfg.k)
+    want_kl, want_dqi = oracle.kl_rows(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], rows, sel, 128, w)
+    assert_grad_close(kl[rows], want_kl, "kl (sampled rows)")
+    assert_grad_close(dqi[rows] / w, want_dqi / w, "dq_idx (sampled rows)")
+    for r in range(cfg.H_kv):
+        s = dki[:, r].sum(axis=0)
+        assert np.max(np.abs(s)) <= 1e-2 * np.abs(dki[:, r]).sum(axis=0).max(), r
+
