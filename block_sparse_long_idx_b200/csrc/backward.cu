@@ -56,8 +56,6 @@ struct BwdCfg {
     static_assert(BASE % 16 == 0, "KL region alignment");
 };
 
-__device__ __forceinline__ uint32_t ld32(const uint16_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
-
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
@@ -274,25 +272,27 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
             cp_async_wait_all();
             __syncthreads();
 
-            // S^T = K_w Q^T and dP^T = V_w dO^T: keys kw0 .. kw0+15 x the 16 rows (two n-tiles)
+            // S^T = K_w Q^T and dP^T = V_w dO^T: keys kw0 .. kw0+15 x the 16 rows (two n-tiles). A
+            // fragments (K_w, V_w rows) and the B fragments of both n-tiles (Q, dO rows) by ldmatrix.x4:
+            // B matrices are (rows 0-7, d 0-7), (rows 0-7, d 8-15), (rows 8-15, d 0-7), (rows 8-15, d 8-15)
             float st[2][4], dpt[2][4];
 #pragma unroll
             for (int n = 0; n < 2; ++n)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) st[n][q] = dpt[n][q] = 0.f;
+            const int a_off = (kw0 + (lane & 15)) * LD + (lane >> 4) * 8;
+            const int b_off = ((lane & 7) + ((lane >> 4) << 3)) * LD + ((lane >> 3) & 1) * 8;
 #pragma unroll
             for (int ks = 0; ks < DH / 16; ++ks) {
-                const int c0 = ks * 16 + 2 * t;
-                const uint32_t ak[4] = {ld32(sK + (kw0 + g) * LD + c0), ld32(sK + (kw0 + g + 8) * LD + c0),
-                                        ld32(sK + (kw0 + g) * LD + c0 + 8), ld32(sK + (kw0 + g + 8) * LD + c0 + 8)};
-                const uint32_t av[4] = {ld32(sV + (kw0 + g) * LD + c0), ld32(sV + (kw0 + g + 8) * LD + c0),
-                                        ld32(sV + (kw0 + g) * LD + c0 + 8), ld32(sV + (kw0 + g + 8) * LD + c0 + 8)};
-#pragma unroll
-                for (int n = 0; n < 2; ++n) {
-                    const int row = n * 8 + g;
-                    mma_bf16_16816(st[n], ak, ld32(sQ + row * LD + c0), ld32(sQ + row * LD + c0 + 8));
-                    mma_bf16_16816(dpt[n], av, ld32(sdO + row * LD + c0), ld32(sdO + row * LD + c0 + 8));
-                }
+                uint32_t ak[4], av[4], bq[4], bo[4];
+                ldmatrix_x4(ak[0], ak[1], ak[2], ak[3], sK + a_off + ks * 16);
+                ldmatrix_x4(av[0], av[1], av[2], av[3], sV + a_off + ks * 16);
+                ldmatrix_x4(bq[0], bq[1], bq[2], bq[3], sQ + b_off + ks * 16);
+                ldmatrix_x4(bo[0], bo[1], bo[2], bo[3], sdO + b_off + ks * 16);
+                mma_bf16_16816(st[0], ak, bq[0], bq[1]);
+                mma_bf16_16816(st[1], ak, bq[2], bq[3]);
+                mma_bf16_16816(dpt[0], av, bo[0], bo[1]);
+                mma_bf16_16816(dpt[1], av, bo[2], bo[3]);
             }
             // P^T and dS^T; element (n, q) is key kw0 + g (+8 for q >= 2), row n*8 + 2t + (q & 1)
 #pragma unroll
@@ -340,9 +340,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
                 for (int q = 0; q < 4; ++q) dq[n][q] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < kBk / 16; ++ks) {
-                const int c0 = ks * 16 + 2 * t;
-                const uint32_t af[4] = {ld32(sdS + g * LDS + c0), ld32(sdS + (g + 8) * LDS + c0),
-                                        ld32(sdS + g * LDS + c0 + 8), ld32(sdS + (g + 8) * LDS + c0 + 8)};
+                uint32_t af[4];
+                ldmatrix_x4(af[0], af[1], af[2], af[3], sdS + (lane & 15) * LDS + (lane >> 4) * 8 + ks * 16);
 #pragma unroll
                 for (int n = 0; n < NQT; ++n) {
                     uint32_t b0, b1;
@@ -389,14 +388,21 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_attn_kernel(BwdArgs a)
                     }
                 }
                 __syncthreads();
-                // dq_idx of each position: sum over the block's keys of w (P_idx - P) k_idx
-                for (int c = tid; c < PPT * DI; c += kBwdWarps * 32) {
-                    const int pl = c / DI, d = c % DI;
+                // dq_idx of each position: sum over the block's keys of w (P_idx - P) k_idx, each output
+                // split over PARTS key ranges so that all threads share the work
+                constexpr int OUT = PPT * DI;
+                constexpr int PARTS = OUT >= kBwdWarps * 32 ? 1 : kBwdWarps * 32 / OUT;
+                constexpr int KPP = kBk / PARTS;
+                static_assert(kBk % PARTS == 0, "key ranges");
+                for (int c = tid; c < OUT * PARTS; c += kBwdWarps * 32) {
+                    const int o = c % OUT, part = c / OUT;
+                    const int pl = o / DI, d = o % DI;
                     const int pos = sPos[pl * G];
                     if (pos < 0) continue;
                     float acc = 0.f;
 #pragma unroll 8
-                    for (int jj = 0; jj < kBk; ++jj) acc = fmaf(sG[pl * kBk + jj], sKI[jj * LDI + d], acc);
+                    for (int jj = part * KPP; jj < (part + 1) * KPP; ++jj)
+                        acc = fmaf(sG[pl * kBk + jj], sKI[jj * LDI + d], acc);
                     atomicAdd(a.dqi_acc + ((int64_t)pos * a.H_kv + r) * DI + d, acc);
                 }
             }

@@ -23,6 +23,16 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Four 8x8 b16 matrices; lanes 8i .. 8i+7 give the row addresses of matrix i, which lands in ri.
+// For an A fragment of a row-major 16 x 16 block at p0 (row stride ld): lane address
+// p0 + (lane % 16) * ld + (lane / 16) * 8 gives r0..r3 = a0..a3.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, const void* p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(p)));
+}
+
 // B fragment of a k x n block stored k-major in shared memory (row = k, 8 consecutive n per row):
 // lanes 0-15 give the addresses of rows k0 .. k0+15 at column n0.
 __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, const void* p)
