@@ -106,6 +106,16 @@ def test_host_fault_injection():
     env = dict(os.environ, MSA_FAULT_INJECT="msa_index_topk")
     out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert "STATUS 4" in out.stdout, out.stdout + out.stderr
+    # the backward's injection point sits after its argument checks, before anything is enqueued
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "import block_sparse_long_idx_b200 as m\n"
+        "r = m.lib.msa_sparse_backward(%d, %d, %d, %d, %d, %d, 1024, 8, 2, 64, 128, 4, %d, None, None, %d, %d, %d, "
+        "None, None, 0, 1.0, None, None, None, %d, 1 << 40, None)\n"
+        "print('STATUS', r)\n" % (ROOT, P, P, P, P, P2, P, P, P, P, P, WS))
+    env = dict(os.environ, MSA_FAULT_INJECT="msa_sparse_backward")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert "STATUS 4" in out.stdout, out.stdout + out.stderr
 
 
 def test_selftest_validation(msa):
