@@ -63,11 +63,21 @@ class Oracle:
                                                      _int, _c_i32p, _c_i32p, _i64, _c_f64p, _c_f64p, _int]
         L.msa_oracle_kl_rows.argtypes = [_c_u16p, _c_u16p, _c_i64p, _i64, _c_u16p, _c_u16p, _i64, _int, _int, _int,
                                          _int, _int, _int, _c_i32p, ctypes.c_double, _c_f64p, _c_f64p, _int]
+        _c_u8p = ctypes.POINTER(ctypes.c_uint8)
+        L.msa_oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.msa_oracle_e4m3_decode.restype = ctypes.c_double
+        L.msa_oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.msa_oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.msa_oracle_quantize_e4m3_rows.argtypes = [_c_u16p, _i64, _int, _c_u8p, _c_f64p]
+        L.msa_oracle_attend_rows_e4m3.argtypes = [_c_u8p, _c_f64p, _c_i64p, _i64, _c_u8p, _c_f64p, _c_u8p, _c_f64p,
+                                                  _i64, _int, _int, _int, _int, _int, _c_i32p, _c_f64p, _c_f64p,
+                                                  _int]
         L.msa_oracle_kl_dk_idx_blocks.argtypes = [_c_u16p, _c_u16p, _c_u16p, _c_u16p, _i64, _int, _int, _int, _int,
                                                   _int, _int, _c_i32p, _c_i32p, _i64, ctypes.c_double, _c_f64p, _int]
         for f in ("msa_oracle_select_rows", "msa_oracle_kv2q", "msa_oracle_attend_rows", "msa_oracle_decode",
                   "msa_oracle_max_threads", "msa_oracle_backward_dq_rows", "msa_oracle_backward_dkv_blocks",
-                  "msa_oracle_kl_rows", "msa_oracle_kl_dk_idx_blocks"):
+                  "msa_oracle_kl_rows", "msa_oracle_kl_dk_idx_blocks", "msa_oracle_quantize_e4m3_rows",
+                  "msa_oracle_attend_rows_e4m3"):
             getattr(L, f).restype = _int
         self.L = L
 
@@ -257,6 +267,48 @@ class Oracle:
             raise ValueError("msa_oracle_kl_dk_idx_blocks: bad arguments")
         return g
 
+    # ------------------------------------------------------------------ FP8 (E4M3) main branch
+    def e4m3_decode(self, code: int) -> float:
+        return float(self.L.msa_oracle_e4m3_decode(code))
+
+    def e4m3_encode(self, x: float) -> int:
+        return int(self.L.msa_oracle_e4m3_encode(float(x)))
+
+    def quantize_e4m3(self, x):
+        """Per-row E4M3 quantisation of a bf16 tensor [..., cols]: (codes uint8 same shape, scales f64 [...])."""
+        xs = _u16(x)
+        rows = int(np.prod(xs.shape[:-1]))
+        codes = np.empty(xs.shape, dtype=np.uint8)
+        scales = np.empty(xs.shape[:-1], dtype=np.float64)
+        rc = self.L.msa_oracle_quantize_e4m3_rows(_p(xs, _c_u16p), rows, xs.shape[-1],
+                                                  codes.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                                  _p(scales, _c_f64p))
+        if rc:
+            raise ValueError("msa_oracle_quantize_e4m3_rows: bad arguments")
+        return codes, scales
+
+    def attend_rows_e4m3(self, q8, k8, v8, rows, sel, B_k: int, n_threads: int = 0):
+        """Sparse attention on E4M3 inputs; q8/k8/v8 = (codes, scales) from quantize_e4m3 of q [N, H_q, d_h],
+        k/v [N, H_kv, d_h]. Returns (out f64 [n, H_q, d_h], lse f64 [n, H_q])."""
+        (qc, qs), (kc, ks), (vc, vs) = q8, k8, v8
+        N, H_kv, d_h = kc.shape
+        H_q = qc.shape[1]
+        k = sel.shape[2]
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        u8 = ctypes.POINTER(ctypes.c_uint8)
+        qg, qsg = np.ascontiguousarray(qc[rows]), np.ascontiguousarray(qs[rows])
+        kc, ks, vc, vs = (np.ascontiguousarray(a) for a in (kc, ks, vc, vs))
+        sel = np.ascontiguousarray(sel, dtype=np.int32)
+        out = np.empty((len(rows), H_q, d_h), dtype=np.float64)
+        lse = np.empty((len(rows), H_q), dtype=np.float64)
+        rc = self.L.msa_oracle_attend_rows_e4m3(qg.ctypes.data_as(u8), _p(qsg, _c_f64p), _p(rows, _c_i64p), len(rows),
+                                                kc.ctypes.data_as(u8), _p(ks, _c_f64p), vc.ctypes.data_as(u8),
+                                                _p(vs, _c_f64p), N, H_q, H_kv, d_h, B_k, k, _p(sel, _c_i32p),
+                                                _p(out, _c_f64p), _p(lse, _c_f64p), n_threads)
+        if rc:
+            raise ValueError("msa_oracle_attend_rows_e4m3: bad arguments")
+        return out, lse
+
 
 _default = None
 
@@ -310,6 +362,14 @@ def kl_rows(*a, **kw):
 
 def kl_dk_idx_blocks(*a, **kw):
     return default().kl_dk_idx_blocks(*a, **kw)
+
+
+def quantize_e4m3(*a, **kw):
+    return default().quantize_e4m3(*a, **kw)
+
+
+def attend_rows_e4m3(*a, **kw):
+    return default().attend_rows_e4m3(*a, **kw)
 
 
 def max_threads() -> int:

@@ -28,6 +28,7 @@
  *  (4) Decode: (1)+(3) for the single query at position len-1 of each cached sequence.
  *  (5) Main Branch backward: the gradient of (3) in q, k and v with the selected sets fixed.
  *  (6) Index Branch KL alignment loss (explainer section 03) and its gradient in q_idx, k_idx.
+ *  (7) FP8 main branch: E4M3 quantisation of q, k, v per row and (3) on the dequantised values.
  *
  * Inputs are bf16 bit patterns widened exactly to double. All sums are in double.
  */
@@ -684,5 +685,152 @@ int msa_oracle_kl_dk_idx_blocks(const uint16_t* q, const uint16_t* q_idx, const 
         free(p);
         free(tok);
     }
+    return err;
+}
+
+/* ---------------------------------------------------------------------------------------- */
+/* (7) FP8 main branch: OCP E4M3 quantisation and attention over the dequantised values.      */
+/* ---------------------------------------------------------------------------------------- */
+/*
+ * The blog page's kernel paragraph says the kernels were tuned on FP8 tensor cores but gives no
+ * quantisation. Reading: q, k and v are quantised to E4M3 (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, subnormals, no infinities, largest finite 448, S.1111.111 is NaN) row by row,
+ * one scale per (token, head) row = amax / 448, round to nearest with ties to the even code,
+ * saturating at 448; the main branch (3) then runs on the dequantised values code * scale.
+ */
+
+double msa_oracle_e4m3_decode(uint8_t c)
+{
+    if ((c & 0x7F) == 0x7F) return NAN; /* S.1111.111 */
+    const int e = (c >> 3) & 15, m = c & 7;
+    const double v = e == 0 ? ldexp((double)m, -9)         /* subnormal: m/8 * 2^-6 */
+                            : ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+    return (c & 0x80) ? -v : v;
+}
+
+/* nearest finite E4M3 value by search over the 127 non-negative finite codes (0x00..0x7E, which
+ * decode in increasing order); ties go to the code with an even mantissa; |x| >= 448 saturates */
+uint8_t msa_oracle_e4m3_encode(double x)
+{
+    const uint8_t sign = signbit(x) ? 0x80 : 0;
+    const double a = fabs(x);
+    uint8_t best = 0;
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double dc = fabs(msa_oracle_e4m3_decode((uint8_t)c) - a);
+        const double db = fabs(msa_oracle_e4m3_decode(best) - a);
+        if (dc < db || (dc == db && (c & 1) == 0)) best = (uint8_t)c;
+    }
+    return sign | best;
+}
+
+/*
+ *   x      : [rows, cols] bf16
+ *   codes  : [rows, cols] E4M3 codes;  scales : [rows] (amax / 448; 1 for an all-zero row)
+ */
+int msa_oracle_quantize_e4m3_rows(const uint16_t* x, int64_t rows, int cols, uint8_t* codes, double* scales)
+{
+    if (!x || !codes || !scales || rows < 0 || cols < 1) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        double amax = 0.0;
+        for (int c = 0; c < cols; ++c) {
+            const double v = fabs(bf16_to_double(x[r * cols + c]));
+            if (v > amax) amax = v;
+        }
+        const double scale = amax > 0.0 ? amax / 448.0 : 1.0;
+        scales[r] = scale;
+        for (int c = 0; c < cols; ++c) codes[r * cols + c] = msa_oracle_e4m3_encode(bf16_to_double(x[r * cols + c]) / scale);
+    }
+    return 0;
+}
+
+/* (3) for one (i, h) on double inputs (the dequantised rows) */
+static void attend_one_f64(const double* q, const double* kseq, const double* vseq, int64_t i, int r, int H_kv,
+                           int d_h, int B_k, int k, const int32_t* sel, double* out, double* lse, double* logits)
+{
+    const double scale = 1.0 / sqrt((double)d_h);
+    int64_t n = 0;
+    double m = -INFINITY;
+    for (int s = 0; s < k; ++s) {
+        const int32_t b = sel[s];
+        if (b < 0) continue;
+        for (int64_t j = (int64_t)b * B_k; j < ((int64_t)b + 1) * B_k && j <= i; ++j) {
+            const double* kr = kseq + ((size_t)j * H_kv + r) * d_h;
+            double dot = 0.0;
+            for (int d = 0; d < d_h; ++d) dot += q[d] * kr[d];
+            logits[n] = dot * scale;
+            if (logits[n] > m) m = logits[n];
+            ++n;
+        }
+    }
+    double z = 0.0;
+    for (int d = 0; d < d_h; ++d) out[d] = 0.0;
+    n = 0;
+    for (int s = 0; s < k; ++s) {
+        const int32_t b = sel[s];
+        if (b < 0) continue;
+        for (int64_t j = (int64_t)b * B_k; j < ((int64_t)b + 1) * B_k && j <= i; ++j) {
+            const double p = exp(logits[n++] - m);
+            z += p;
+            const double* vr = vseq + ((size_t)j * H_kv + r) * d_h;
+            for (int d = 0; d < d_h; ++d) out[d] += p * vr[d];
+        }
+    }
+    for (int d = 0; d < d_h; ++d) out[d] /= z;
+    *lse = m + log(z);
+}
+
+/*
+ * (3) on E4M3 inputs: value = code * scale of its row.
+ *   qc, qs : [n_rows, H_q, d_h] codes, [n_rows, H_q] scales of the requested rows (gathered)
+ *   kc, ks, vc, vs : [N, H_kv, d_h] codes, [N, H_kv] scales
+ *   sel    : [n_rows, H_kv, k];  out : [n_rows, H_q, d_h] double;  lse : [n_rows, H_q] double
+ */
+int msa_oracle_attend_rows_e4m3(const uint8_t* qc, const double* qs, const int64_t* rows, int64_t n_rows,
+                                const uint8_t* kc, const double* ks, const uint8_t* vc, const double* vs, int64_t N,
+                                int H_q, int H_kv, int d_h, int B_k, int k, const int32_t* sel, double* out,
+                                double* lse, int n_threads)
+{
+    if (!qc || !qs || !rows || !kc || !ks || !vc || !vs || !sel || !out || !lse || H_kv < 1 || H_q % H_kv ||
+        d_h < 1 || d_h > 512)
+        return -1;
+    for (int64_t t = 0; t < n_rows; ++t)
+        if (rows[t] < 0 || rows[t] >= N) return -1;
+    const int G = H_q / H_kv;
+    double* kd = (double*)malloc(sizeof(double) * (size_t)N * H_kv * d_h);
+    double* vd = (double*)malloc(sizeof(double) * (size_t)N * H_kv * d_h);
+    if (!kd || !vd) {
+        free(kd);
+        free(vd);
+        return -1;
+    }
+    for (int64_t x = 0; x < N * H_kv; ++x)
+        for (int d = 0; d < d_h; ++d) {
+            kd[x * d_h + d] = msa_oracle_e4m3_decode(kc[x * d_h + d]) * ks[x];
+            vd[x * d_h + d] = msa_oracle_e4m3_decode(vc[x * d_h + d]) * vs[x];
+        }
+    set_threads(n_threads);
+    int err = 0;
+#pragma omp parallel
+    {
+        double* logits = (double*)malloc(sizeof(double) * (size_t)k * B_k);
+        if (!logits) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1) collapse(2)
+        for (int64_t t = 0; t < n_rows; ++t)
+            for (int h = 0; h < H_q; ++h)
+                if (logits) {
+                    double qd[512];
+                    const size_t qh = (size_t)t * H_q + h;
+                    for (int d = 0; d < d_h; ++d) qd[d] = msa_oracle_e4m3_decode(qc[qh * d_h + d]) * qs[qh];
+                    const int r = h / G;
+                    attend_one_f64(qd, kd, vd, rows[t], r, H_kv, d_h, B_k, k, sel + ((size_t)t * H_kv + r) * k,
+                                   out + qh * d_h, lse + qh, logits);
+                }
+        free(logits);
+    }
+    free(kd);
+    free(vd);
     return err;
 }

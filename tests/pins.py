@@ -405,6 +405,81 @@ def check_kl_uniform_teacher_closed_form(o):
     assert np.max(np.abs(kl)) < 1e-14 and np.max(np.abs(dqi)) < 1e-14 and np.max(np.abs(dki)) < 1e-14
 
 
+# ------------------------------------------------------------------------------- FP8 (E4M3)
+
+def check_e4m3_codec_closed_form(o):
+    """E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals, no infinities, 448 the
+    largest finite, S.1111.111 NaN): values from the format's definition, round trip of every finite
+    code, ties to the even mantissa, saturation."""
+    pos = [o.e4m3_decode(c) for c in range(0x7F)]
+    assert pos[0] == 0.0 and pos[1] == 2.0 ** -9 and pos[7] == 7 * 2.0 ** -9     # subnormals m * 2^-9
+    assert pos[8] == 2.0 ** -6 and pos[0x7E] == 448.0 == 1.75 * 2 ** 8           # smallest normal, largest
+    assert all(b > a for a, b in zip(pos, pos[1:]))                               # increasing
+    assert math.isnan(o.e4m3_decode(0x7F)) and math.isnan(o.e4m3_decode(0xFF))
+    for c in list(range(0x7F)) + list(range(0x80, 0xFF)):
+        assert o.e4m3_decode(c) == (-1.0 if c & 0x80 else 1.0) * pos[c & 0x7F]
+        assert o.e4m3_encode(o.e4m3_decode(c)) == c, hex(c)
+    # hand-worked: 0.1 lies in [2^-4, 2^-3), step 2^-7, 0.1 / 2^-7 = 12.8 -> 13 * 2^-7 = 1.625 * 2^-4:
+    # exponent field 3, mantissa 5 -> 0x1D; 3 = 1.5 * 2^1 -> 0x44; 300 in [256, 512), step 32: 288 is
+    # nearer than 320 -> 1.125 * 2^8 -> 0x79; 2^-10 is halfway between 0 and 2^-9 -> the even code 0x00
+    assert o.e4m3_encode(0.1) == 0x1D and o.e4m3_decode(0x1D) == 0.1015625
+    assert o.e4m3_encode(3.0) == 0x44 and o.e4m3_encode(-3.0) == 0xC4
+    assert o.e4m3_encode(300.0) == 0x79 and o.e4m3_decode(0x79) == 288.0
+    assert o.e4m3_encode(2.0 ** -10) == 0x00 and o.e4m3_encode(3 * 2.0 ** -10) == 0x02   # 1.5 -> 2 (even)
+    assert o.e4m3_encode(1e9) == 0x7E and o.e4m3_encode(-1e9) == 0xFE and o.e4m3_encode(-0.0) == 0x80
+    for c in range(0x08, 0x7E):                                                   # midpoints of normals
+        mid = 0.5 * (pos[c] + pos[c + 1])
+        assert o.e4m3_encode(mid) == (c if c % 2 == 0 else c + 1), hex(c)
+
+
+def check_e4m3_quantize_rows(o):
+    """Per-row scale amax / 448: each row's largest magnitude becomes +-448, and every value is
+    within half a step of the format (relative 2^-4 in the normal range) after dequantisation."""
+    x = normal_bf16((50, 4, 32), 31, "e4m3")
+    codes, scales = o.quantize_e4m3(x)
+    X = bf16_bits_to_f64(x)
+    amax = np.abs(X).max(axis=-1)
+    assert np.array_equal(scales, amax / 448.0)
+    deq = np.vectorize(o.e4m3_decode)(codes) * scales[..., None]
+    top = np.abs(X) == amax[..., None]
+    assert np.all(np.abs(codes[top] & 0x7F) == 0x7E)
+    rel = np.abs(X) / scales[..., None]
+    normal = rel >= 2.0 ** -6
+    assert np.all(np.abs(deq - X)[normal] <= 2.0 ** -4 * np.abs(X)[normal])
+    assert np.all(np.abs(deq - X)[~normal] <= 2.0 ** -10 * np.broadcast_to(scales[..., None], X.shape)[~normal])
+
+
+def _e4m3_case(o, N, H_q, H_kv, d_h, seed):
+    inp = _attn_inputs(N, H_q, H_kv, d_h, 8, seed)
+    q8, k8, v8 = (o.quantize_e4m3(inp[n]) for n in ("q", "k", "v"))
+    dec = np.vectorize(o.e4m3_decode)
+    deq = [dec(c) * s[..., None] for c, s in (q8, k8, v8)]
+    return inp, (q8, k8, v8), deq
+
+
+def check_attention_e4m3_dense_invariant(o):
+    """FP8 main branch with k*B_k >= N: textbook dense causal GQA attention on the dequantised q, k, v."""
+    N, H_q, H_kv, d_h, B_k, k = 80, 4, 2, 16, 16, 5
+    inp, (q8, k8, v8), (Q, K, V) = _e4m3_case(o, N, H_q, H_kv, d_h, 41)
+    rows = np.arange(N)
+    sel = o.select_rows(inp["q_idx"], inp["k_idx"], rows, B_k, k)
+    out, lse = o.attend_rows_e4m3(q8, k8, v8, rows, sel, B_k)
+    want, want_lse = ref.dense_causal_gqa_f64(Q, K, V)
+    assert np.max(np.abs(out - want)) < 1e-12 and np.max(np.abs(lse - want_lse)) < 1e-12
+
+
+def check_attention_e4m3_masked_bruteforce(o):
+    """FP8 main branch with k*B_k < N: dense attention under the selection mask on the dequantised values."""
+    N, H_q, H_kv, d_h, B_k, k = 150, 4, 2, 16, 16, 3
+    inp, (q8, k8, v8), (Q, K, V) = _e4m3_case(o, N, H_q, H_kv, d_h, 42)
+    rows = np.arange(N)
+    sel = o.select_rows(inp["q_idx"], inp["k_idx"], rows, B_k, k)
+    out, lse = o.attend_rows_e4m3(q8, k8, v8, rows, sel, B_k)
+    allowed = ref.selection_mask(np.ascontiguousarray(sel.transpose(1, 0, 2)), N, B_k)
+    want, want_lse = ref.masked_attention_f64(Q, K, V, allowed)
+    assert np.max(np.abs(out - want)) < 1e-12 and np.max(np.abs(lse - want_lse)) < 1e-12
+
+
 ALL_CHECKS = [
     check_selection_bruteforce,
     check_selection_ties_closed_form,
@@ -425,4 +500,8 @@ ALL_CHECKS = [
     check_backward_dv_sums_to_dout,
     check_kl_autograd,
     check_kl_uniform_teacher_closed_form,
+    check_e4m3_codec_closed_form,
+    check_e4m3_quantize_rows,
+    check_attention_e4m3_dense_invariant,
+    check_attention_e4m3_masked_bruteforce,
 ]

@@ -37,7 +37,11 @@ def dense_selection(q_idx, k_idx, B_k: int, k: int) -> np.ndarray:
 
 def dense_causal_gqa(q, kk, v):
     """Dense causal GQA attention in float64. Returns (out [N, H_q, d_h], lse [N, H_q])."""
-    Q, K, V = bf16_bits_to_f64(q), bf16_bits_to_f64(kk), bf16_bits_to_f64(v)
+    return dense_causal_gqa_f64(bf16_bits_to_f64(q), bf16_bits_to_f64(kk), bf16_bits_to_f64(v))
+
+
+def dense_causal_gqa_f64(Q, K, V):
+    """dense_causal_gqa on float64 arrays."""
     N, H_q, d_h = Q.shape
     H_kv = K.shape[1]
     G = H_q // H_kv
@@ -58,7 +62,11 @@ def dense_causal_gqa(q, kk, v):
 
 def masked_attention(q, kk, v, allowed):
     """Attention with an explicit boolean mask allowed[h_group, i, j]. float64."""
-    Q, K, V = bf16_bits_to_f64(q), bf16_bits_to_f64(kk), bf16_bits_to_f64(v)
+    return masked_attention_f64(bf16_bits_to_f64(q), bf16_bits_to_f64(kk), bf16_bits_to_f64(v), allowed)
+
+
+def masked_attention_f64(Q, K, V, allowed):
+    """masked_attention on float64 arrays."""
     N, H_q, d_h = Q.shape
     H_kv = K.shape[1]
     G = H_q // H_kv

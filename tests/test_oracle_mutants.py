@@ -34,8 +34,11 @@ MUTANTS = [
     ("local_block_not_forced", "sel[n++] = (int32_t)local;", "if (take < k) sel[n++] = (int32_t)(local > 0 ? local - 1 : 0);"),
     ("scale_1_over_d", "const double scale = 1.0 / sqrt((double)d_h);\n    double q[512];",
      "const double scale = 1.0 / (double)d_h;\n    double q[512];"),
-    ("bwd_logits_scale_1_over_d", "const double scale = 1.0 / sqrt((double)d_h);\n    int64_t n = 0;",
-     "const double scale = 1.0 / (double)d_h;\n    int64_t n = 0;"),
+    ("bwd_logits_scale_1_over_d",
+     "const double scale = 1.0 / sqrt((double)d_h);\n    int64_t n = 0;\n    double m = -INFINITY;\n"
+     "    for (int s = 0; s < k; ++s) {\n        int32_t b",
+     "const double scale = 1.0 / (double)d_h;\n    int64_t n = 0;\n    double m = -INFINITY;\n"
+     "    for (int s = 0; s < k; ++s) {\n        int32_t b"),
     ("causal_strict", "j <= i; ++j) {\n            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;\n            double dot = 0.0;\n            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);\n            logits[n]",
      "j < i; ++j) {\n            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;\n            double dot = 0.0;\n            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);\n            logits[n]"),
     ("bwd_causal_strict", "j <= i; ++j) {\n            const uint16_t* kr = kseq + ((size_t)j * H_kv + r) * d_h;\n            double dot = 0.0;\n            for (int d = 0; d < d_h; ++d) dot += q[d] * bf16_to_double(kr[d]);\n            p[n]",
@@ -48,7 +51,8 @@ MUTANTS = [
      "const int r = h % H_kv;\n                    attend_one("),
     ("bwd_wrong_gqa_group", "const int r = h / G;\n                    double qd[512], dod[512];",
      "const int r = h % H_kv;\n                    double qd[512], dod[512];"),
-    ("lse_missing_max", "*lse = m + log(z);", "*lse = log(z);"),
+    ("lse_missing_max", "*lse = m + log(z);\n}\n\n/*\n *   q    :", "*lse = log(z);\n}\n\n/*\n *   q    :"),
+    ("e4m3_lse_missing_max", "*lse = m + log(z);\n}\n\n/*\n * (3) on E4M3", "*lse = log(z);\n}\n\n/*\n * (3) on E4M3"),
     ("kv2q_slot_off_by_one", "ent[fill[b]++] = (int32_t)(i * k + s);", "ent[fill[b]++] = (int32_t)(i * k + s + 1);"),
     ("bwd_softmax_jacobian_without_D", "ds[t] = p[t] * (dp - D);", "ds[t] = p[t] * dp;"),
     ("bwd_dk_from_dout", "gk[jj * d_h + d] += scale * ds[u] * qd[d];", "gk[jj * d_h + d] += scale * ds[u] * dod[d];"),
@@ -60,6 +64,11 @@ MUTANTS = [
     ("kl_gradient_sign", "const double gs = w * (exp(lq[u]) - P[u]);\n                        const uint16_t* kr",
      "const double gs = w * (P[u] - exp(lq[u]));\n                        const uint16_t* kr"),
     ("kl_student_scaled", "lq[t] = s;\n", "lq[t] = s / sqrt((double)d_idx);\n"),
+    ("e4m3_ties_to_odd", "(dc == db && (c & 1) == 0)", "(dc == db && (c & 1) == 1)"),
+    ("e4m3_exponent_bias_8", "ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 11)"),
+    ("e4m3_scale_over_240", "amax > 0.0 ? amax / 448.0 : 1.0", "amax > 0.0 ? amax / 240.0 : 1.0"),
+    ("e4m3_value_scale_dropped", "kd[x * d_h + d] = msa_oracle_e4m3_decode(kc[x * d_h + d]) * ks[x];",
+     "kd[x * d_h + d] = msa_oracle_e4m3_decode(kc[x * d_h + d]);"),
 ]
 
 
