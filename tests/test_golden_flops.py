@@ -39,3 +39,14 @@ def test_main_branch_budget_is_linear_in_n():
     a = roofline.main_branch_flops(2 ** 17, 64, 128, 16, 128)
     b = roofline.main_branch_flops(2 ** 20, 64, 128, 16, 128)
     assert b / a == 8.0
+
+
+def test_backward_flops_are_five_products():
+    """Backward with the selections fixed: per (row, head, selected block) the recomputed S and the
+    dP, dV, dK, dQ products, five B_k x d_h contractions of 2 FLOP per multiply-add against the
+    forward's two."""
+    N, H_q, d_h, k, B_k = 2 ** 17, 64, 128, 16, 128
+    per_unit = 5 * 2 * B_k * d_h
+    assert roofline.main_branch_backward_flops(N, H_q, d_h, k, B_k) == per_unit * N * H_q * k
+    assert roofline.main_branch_backward_flops(N, H_q, d_h, k, B_k) == 2.5 * roofline.main_branch_flops(N, H_q, d_h,
+                                                                                                          k, B_k)
