@@ -45,6 +45,7 @@ def parse_args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch (varlen) prefill leg")
     ap.add_argument("--no-backward", action="store_true", help="skip the main-branch backward leg")
+    ap.add_argument("--no-long", action="store_true", help="skip the 1M-token prefill leg")
     ap.add_argument("--decode-workload", default=synth.DECODE64.name, choices=sorted(synth.DECODE_CONFIGS))
     ap.add_argument("--e2e-steps", type=int, default=8,
                     help="pipelined host-buffer steps (the first input copy and the last output copy are not overlapped)")
@@ -69,9 +70,11 @@ def load_peaks():
 # measured on: after any change to them the bench reports traffic as null.
 PROFILED_TRAFFIC = {
     "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "94f46dc3167c3d8e",
-             "bytes_per_row": 308058.5, "capture": "profiles/sparse_attn_prefill_N32768.md (8192-row pass)"},
+             "bytes_per_row": 308058.5,
+             "capture": "ncu capture of sparse_attn_kernel<128, 16> on the N=32768 prefill, one 8192-row pass"},
     "combine": {"files": ("combine.cu", "common.cuh", "sm100.cuh"), "sha256_16": "efedf33b948eb033",
-                "bytes_per_row": 282506.7, "capture": "profiles/combine_prefill_N32768.md (8192-row pass)"},
+                "bytes_per_row": 282506.7,
+                "capture": "ncu capture of combine_kernel on the N=32768 prefill, one 8192-row pass"},
 }
 
 
@@ -234,6 +237,100 @@ class ClockSampler:
                 "sm_min_mhz": min(sm) if sm else None,
                 "sm_max_mhz": self.samples[-1][1] if self.samples else None, "reasons": reasons,
                 "samples": len(sm), "source": "nvml" if self.proc is None else "nvidia-smi"}
+
+
+def kernel_stats(kern, steps, cfg, peaks, dec_bytes=None):
+    """Per-kernel time per step and roofline fraction from the traced CUDA-event durations:
+    achieved = algorithmic FLOPs or bytes of the kernel per step / its time per step."""
+    N, H_q, H_kv, d_h, d_idx, k, B_k = cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.d_idx, cfg.k, cfg.B_k
+    algo = {"index_topk": ("tensor", roofline.index_branch_flops(N, H_kv, d_idx)),
+            "attn": ("tensor", roofline.main_branch_flops(N, H_q, d_h, k, B_k)),
+            "combine": ("hbm", roofline.combine_bytes(N, H_q, H_kv, d_h, k, B_k)),
+            "kv2q": ("hbm", roofline.kv2q_bytes(N, H_kv, k, B_k))}
+    if dec_bytes:
+        algo["dec_pool"] = ("hbm", dec_bytes["dec_pool"])
+        algo["dec_attn"] = ("hbm", dec_bytes["dec_attn"])
+    kstats = {}
+    for name, durs in kern.items():
+        per_step = sum(durs) / steps
+        ent = {"ms_per_step": per_step, "launches_per_step": len(durs) / steps}
+        if name in algo:
+            bound, work = algo[name]
+            if bound == "tensor":
+                ach = work / (per_step / 1000.0) / 1e12
+                ent.update({"bound": "tensor", "achieved": ach, "unit": "TFLOP/s", "peak": peaks["bf16_tflops"],
+                            "frac": ach / peaks["bf16_tflops"], "algorithmic": work})
+            else:
+                ach = work / (per_step / 1000.0) / 1e9
+                ent.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                            "frac": ach / peaks["hbm_gbs"], "algorithmic": work})
+        if name in ("attn", "combine"):
+            rows = N / max(1.0, ent["launches_per_step"])
+            tr = profiled_traffic(name, rows)
+            ent["traffic"] = tr
+            if tr is not None:
+                ent["traffic_source"] = PROFILED_TRAFFIC[name]["capture"] + ", scaled by rows per launch"
+        kstats[name] = ent
+    return kstats
+
+
+def long_prefill_leg(args, rank, world, dev, peaks, flush):
+    """Prefill of one 1M-token sequence (8192 KV blocks; i.i.d. inputs as at 32K) in passes of 131072
+    query rows: the long-context regime where the index branch's quadratic term dominates."""
+    import torch
+
+    import block_sparse_long_idx_b200 as msa
+
+    cfg = synth.P1M.with_(seed=replicas.replica_seed(synth.P1M.seed, rank))
+    host = synth.prefill_inputs(cfg)
+    t = {n: torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev) for n, a in host.items()}
+    del host
+    N, H_q, H_kv, d_h, k = cfg.N, cfg.H_q, cfg.H_kv, cfg.d_h, cfg.k
+    rows_pass = 131072
+    block_idx = torch.empty((H_kv, N, k), dtype=torch.int32, device=dev)
+    L = msa.msa_kv2q_layout_get(N, H_kv, cfg.B_k, k)
+    kv = msa.KV2Q(L, torch.empty(L.total_bytes, dtype=torch.uint8, device=dev))
+    ws_kv = torch.empty(msa.api.lib.msa_build_kv2q_workspace_size(msa.api.ctypes.byref(L)), dtype=torch.uint8,
+                        device=dev)
+    ws_pf = torch.empty(msa.msa_sparse_prefill_workspace_size(N, H_q, H_kv, d_h, cfg.B_k, k, rows_pass),
+                        dtype=torch.uint8, device=dev)
+    ws_idx = torch.empty(256, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(t["q"])
+    lse = torch.empty((N, H_q), dtype=torch.float32, device=dev)
+
+    def step():
+        cur = torch.cuda.current_stream()
+        msa.msa_index_topk(t["q_idx"], t["k_idx"], cfg.B_k, k, block_idx=block_idx, workspace=ws_idx, stream=cur)
+        msa.api._check("msa_build_kv2q", msa.api.lib.msa_build_kv2q(
+            block_idx.data_ptr(), msa.api.ctypes.byref(L), kv.buf.data_ptr(), ws_kv.data_ptr(), ws_kv.numel(),
+            cur.cuda_stream))
+        msa.msa_sparse_prefill(t["q"], t["k"], t["v"], block_idx, kv, out=out, lse=lse, workspace=ws_pf, stream=cur)
+
+    steps = max(1, min(args.steps, 3))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for ws in (ws_idx, ws_kv, ws_pf):
+        if msa.msa_get_device_error(ws) != 0:
+            raise RuntimeError("device error in the 1M prefill warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    trace = msa.KernelTrace(64 * steps)
+    with trace:
+        for st in range(steps):
+            flush.zero_()
+            ev[st][0].record()
+            step()
+            ev[st][1].record()
+    torch.cuda.synchronize()
+    (ms,) = replicas.max_over_ranks([sum(a.elapsed_time(b) for a, b in ev)], device=dev)
+    res = {"workload": cfg.name, "value": replicas.aggregate_rate(N * steps, world, ms / 1000.0), "unit": UNIT,
+           "ms_per_step": ms / steps, "steps": steps, "rows_per_pass": rows_pass,
+           "kernels": kernel_stats(trace.durations(), steps, cfg, peaks),
+           "note": "one 1048576-token sequence, i.i.d. inputs; index Top-k, inversion, and attention + combine "
+                   "in passes of 131072 query rows; L2 flushed before each step"}
+    del t, block_idx, kv, ws_kv, ws_pf, ws_idx, out, lse
+    torch.cuda.empty_cache()
+    return res
 
 
 def gpu_arm(args, rank, world):
@@ -502,38 +599,19 @@ def gpu_arm(args, rank, world):
                        "pinned memory and its output back; inputs/outputs double-buffered on the device so the "
                        "copies of neighbouring steps overlap the current step's kernels"}
 
+    # 1M-token prefill (passes of 131072 rows): release the 128K workload's large buffers first
+    long_prefill = None
+    if not args.no_long:
+        ws_pf = dt = dev_in = dev_out = pin = out_h = None  # noqa: F841 (drop the 128K buffers)
+        torch.cuda.empty_cache()
+        long_prefill = long_prefill_leg(args, rank, world, dev, peaks, flush)
+
     if rank != 0:
         return
     value = replicas.aggregate_rate(N * args.steps, world, pf_total / 1000.0)
-    kstats = {}
-    fl_main = roofline.main_branch_flops(N, H_q, d_h, k, cfg.B_k)
-    fl_idx = roofline.index_branch_flops(N, H_kv, d_idx)
-    algo = {"index_topk": ("tensor", fl_idx), "attn": ("tensor", fl_main),
-            "combine": ("hbm", roofline.combine_bytes(N, H_q, H_kv, d_h, k, cfg.B_k))}
-    if dcfg:
-        db = roofline.decode_bytes(dh["lens"], dcfg.H_q, dcfg.H_kv, dcfg.d_h, dcfg.d_idx, dcfg.k, dcfg.B_k)
-        algo["dec_pool"] = ("hbm", db["dec_pool"])
-        algo["dec_attn"] = ("hbm", db["dec_attn"])
-    for name, durs in kern.items():
-        per_step = sum(durs) / args.steps
-        ent = {"ms_per_step": per_step, "launches_per_step": len(durs) / args.steps}
-        if name in algo:
-            bound, work = algo[name]
-            if bound == "tensor":
-                ach = work / (per_step / 1000.0) / 1e12
-                ent.update({"bound": "tensor", "achieved": ach, "unit": "TFLOP/s", "peak": peaks["bf16_tflops"],
-                            "frac": ach / peaks["bf16_tflops"], "algorithmic": work})
-            else:
-                ach = work / (per_step / 1000.0) / 1e9
-                ent.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "peak": peaks["hbm_gbs"],
-                            "frac": ach / peaks["hbm_gbs"], "algorithmic": work})
-        if name in ("attn", "combine"):
-            rows = N / max(1.0, ent["launches_per_step"])
-            tr = profiled_traffic(name, rows)
-            ent["traffic"] = tr
-            if tr is not None:
-                ent["traffic_source"] = PROFILED_TRAFFIC[name]["capture"] + ", scaled by rows per launch"
-        kstats[name] = ent
+    dec_bytes = (roofline.decode_bytes(dh["lens"], dcfg.H_q, dcfg.H_kv, dcfg.d_h, dcfg.d_idx, dcfg.k, dcfg.B_k)
+                 if dcfg else None)
+    kstats = kernel_stats(kern, args.steps, cfg, peaks, dec_bytes)
     # dominant kernel of the prefill step
     dom = max((n for n in ("index_topk", "attn", "combine") if n in kstats), key=lambda n: kstats[n]["ms_per_step"])
     d = kstats[dom]
@@ -550,7 +628,7 @@ def gpu_arm(args, rank, world):
                         "ms_per_step": dec_total / args.steps} if dcfg else None),
             "decode_graph": decode_graph,
             "roofline": roof, "kernels": kstats, "cpu_baseline": cpu_base, "e2e": e2e, "varlen": varlen,
-            "backward": backward,
+            "backward": backward, "long_prefill": long_prefill,
             "gpu_launches": int(launches), "clocks": clocks.summary(), "wall_s_timed": wall}
     print(json.dumps(line), flush=True)
 

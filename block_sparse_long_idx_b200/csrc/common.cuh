@@ -75,6 +75,12 @@ struct Kv2qArgs {
 };
 cudaError_t launch_kv2q(const Kv2qArgs& a, cudaStream_t s);
 size_t kv2q_scan_tmp_bytes(int64_t n, int H_kv);
+// msa_build_kv2q_static: host checks (layout, alignment, scratch size, fault hook), then the launch
+// with the error word and scan partials in a fixed scratch (msa_api.cu).
+msa_status kv2q_static_check(const int32_t* block_idx, const msa_kv2q_layout* L, const void* kv2q,
+                             size_t scratch_bytes);
+msa_status kv2q_static_run(const int32_t* block_idx, const msa_kv2q_layout* L, void* kv2q, void* scratch,
+                           cudaStream_t s);
 
 struct AttnArgs {
     int64_t N;

@@ -161,8 +161,8 @@ __global__ void __launch_bounds__(384, 1)
             }
             // drain: every issued k_idx load has landed before the CTA may exit
             for (int g = gstep - 1; g >= 0 && g >= gstep - C::NST; --g)
-                mbar_wait(&sh.kv_full[g % C::NST], (g / C::NST) & 1, kWaitLimit);
-            if (item_cnt > 0) mbar_wait(&sh.q_full, (item_cnt - 1) & 1, kWaitLimit);
+                drain_wait(&sh.kv_full[g % C::NST], (g / C::NST) & 1, a.err, 7, kWaitLimit);
+            if (item_cnt > 0) drain_wait(&sh.q_full, (item_cnt - 1) & 1, a.err, 8, kWaitLimit);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(384, 1)
                 ++item_cnt;
             }
             tc_commit(&sh.done);
-            mbar_wait(&sh.done, 0, kWaitLimit);
+            drain_wait(&sh.done, 0, a.err, 9, kWaitLimit);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue: pool + Top-k

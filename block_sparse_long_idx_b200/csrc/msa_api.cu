@@ -305,6 +305,34 @@ msa_status msa_build_kv2q(const int32_t* block_idx, const msa_kv2q_layout* L, vo
     return build_kv2q_impl(block_idx, L, kv2q, (int*)workspace, (uint8_t*)workspace + kErrBytes, s);
 }
 
+} // extern "C"
+
+namespace msa {
+
+// Host checks of msa_build_kv2q_static: the same layout validation and fault hook as
+// msa_build_kv2q, with a fixed scratch of scratch_bytes in place of the caller's workspace.
+msa_status kv2q_static_check(const int32_t* block_idx, const msa_kv2q_layout* L, const void* kv2q,
+                             size_t scratch_bytes)
+{
+    if (!block_idx || !L || !kv2q) return MSA_ERR_INVALID_ARG;
+    if (!layout_ok(L) || !aligned(kv2q, 256) || !aligned(block_idx, 4)) return MSA_ERR_INVALID_ARG;
+    if (kErrBytes + kv2q_internal_tmp(*L) > scratch_bytes) return MSA_ERR_WORKSPACE;
+    if (injected("msa_build_kv2q_static")) return MSA_ERR_CUDA;
+    return MSA_OK;
+}
+
+// The inversion with its error word and scan partials in `scratch` (a checked layout).
+msa_status kv2q_static_run(const int32_t* block_idx, const msa_kv2q_layout* L, void* kv2q, void* scratch,
+                           cudaStream_t s)
+{
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(scratch, 0, kErrBytes, s), "clearing the error word")) return st0;
+    return build_kv2q_impl(block_idx, L, kv2q, (int*)scratch, (uint8_t*)scratch + kErrBytes, s);
+}
+
+} // namespace msa
+
+extern "C" {
+
 // ------------------------------------------------------------------------------------ sparse prefill
 static size_t partial_row_bytes(int H_q, int d_h, int k) { return (size_t)k * H_q * ((size_t)d_h * 2 + 4); }
 

@@ -77,7 +77,8 @@ __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity)
 }
 
 // Wait for the phase with the given parity to complete. Gives up after `limit` clock cycles and
-// returns false; every caller turns that into an error status instead of spinning forever.
+// returns false instead of spinning forever; callers record that in the device error word
+// (wait_or_abort, poll_or_abort and drain_wait below do).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit)
 {
     if (mbar_try_wait(bar, parity)) return true;
@@ -266,6 +267,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
         }
     }
     return true;
+}
+
+// Wait used while draining a role's in-flight TMA copies or MMAs before the CTA exits: the wait
+// still ends (bounded), and an expired one records MSA_ERR_TIMEOUT (detail = site) in the error word.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* err, int site, long long limit)
+{
+    if (!mbar_wait(bar, parity, limit) && atomicCAS(err, 0, 5 /* MSA_ERR_TIMEOUT */) == 0) err[1] = site;
 }
 
 // wait_or_abort for the MMA issuer: busy-polls (test_wait) instead of sleeping.

@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(512, 1)
                     }
                 }
                 for (int g = it - 1; g >= 0 && g >= it - 2; --g)
-                    mbar_wait(&sh.kv_full[g & 1], (g >> 1) & 1, kWaitLimit);
+                    drain_wait(&sh.kv_full[g & 1], (g >> 1) & 1, a.err, 40, kWaitLimit);
             }
         } else if (warp == 2) {
             // -------------------------------------------------------- tile scheduler + Q gather
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(512, 1)
             }
             if (lane == 0)
                 for (int g = n_tiles - 1; g >= 0 && g >= n_tiles - NQ; --g)
-                    mbar_wait(&sh.q_full[g % NQ], (g / NQ) & 1, kWaitLimit);
+                    drain_wait(&sh.q_full[g % NQ], (g / NQ) & 1, a.err, 41, kWaitLimit);
         } else if (warp == 1) {
             // -------------------------------------------------------- S issuer: S(t) = Q K^T
             if (lane == 0) {
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(512, 1)
                     TL(2, qt);
                 }
                 tc_commit(&sh.done);
-                mbar_wait(&sh.done, 0, kWaitLimit);
+                drain_wait(&sh.done, 0, a.err, 42, kWaitLimit);
             }
         } else if (warp == 3) {
             // -------------------------------------------------------- PV issuer: O(t) = P(t) V
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(512, 1)
                     TL(3, qt);
                 }
                 tc_commit(&sh.done2);
-                mbar_wait(&sh.done2, 0, kWaitLimit);
+                drain_wait(&sh.done2, 0, a.err, 43, kWaitLimit);
             }
         }
     } else if (wg <= 2) {

@@ -69,3 +69,15 @@ def decode_bytes(lens, H_q: int, H_kv: int, d_h: int, d_idx: int, k: int, B_k: i
         toks = n_full * B_k + (L - loc * B_k)
         attn += H_kv * toks * d_h * 2 * 2
     return {"dec_pool": float(pool), "dec_attn": float(attn)}
+
+
+def kv2q_bytes(N: int, H_kv: int, k: int, B_k: int, window: int = 2048) -> float:
+    """KV->Q inversion (counting sort per query window): the selections are read twice (the count
+    pass and the scatter pass, 4 B per (group, row, slot)), every valid entry is written once (4 B),
+    and the per-(group, block, window) counts, bases and item counts are written and read once
+    (3 x 4 B each)."""
+    nb = (N + B_k - 1) // B_k
+    n_windows = (N + window - 1) // window
+    slots = H_kv * N * k
+    valid = n_selected(N, k, B_k) * H_kv
+    return 8.0 * slots + 4.0 * valid + 12.0 * H_kv * nb * n_windows

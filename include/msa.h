@@ -171,7 +171,11 @@ MSA_API msa_status msa_build_kv2q(const int32_t* block_idx, const msa_kv2q_layou
  *     that loads the library until the process exits. The caller still passes block_idx, the
  *     layout and the kv2q output buffer, exactly as for msa_build_kv2q.
  *   - The first call on a device looks up the array's device address on that device (it must be
- *     the current device); make that first call before any stream capture.
+ *     the current device); make that first call before any stream capture. On every call
+ *     `stream` must belong to the current device (else MSA_ERR_INVALID_ARG): the array's address
+ *     differs between GPUs.
+ *   - The layout is validated exactly as msa_build_kv2q validates it (every field, including nb
+ *     and n_windows, must be what msa_kv2q_layout_get returns); a mismatch is MSA_ERR_INVALID_ARG.
  *   - Layouts whose scratch would exceed 1 MiB are rejected with MSA_ERR_WORKSPACE (every shape
  *     this build supports fits: the scan needs one int32 per 1024 (group, block, window) counters).
  *   - All calls share the one array: calls whose work overlaps on the GPU (other streams, other

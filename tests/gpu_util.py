@@ -37,6 +37,31 @@ def assert_out_close(got: np.ndarray, want: np.ndarray, what: str = "out"):
     return mx, mean
 
 
+class OutErr:
+    """|got - want| over many chunks of one output: max and mean over every value, checked at the end
+    against the same tolerance as assert_out_close."""
+
+    def __init__(self, what: str = "out"):
+        self.what, self.mx, self.total, self.n, self.worst = what, 0.0, 0.0, 0, None
+
+    def update(self, got: np.ndarray, want: np.ndarray, offset=0):
+        assert np.isfinite(got).all(), f"{self.what}: non-finite values"
+        d = np.abs(got - want)
+        m = float(d.max())
+        if m > self.mx:
+            idx = np.unravel_index(int(d.argmax()), d.shape)
+            self.mx, self.worst = m, (idx[0] + offset,) + tuple(idx[1:])
+        self.total += float(d.sum())
+        self.n += d.size
+
+    def check(self):
+        mean = self.total / max(self.n, 1)
+        assert self.mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (
+            f"{self.what}: max |d| = {self.mx:.3e} (<= {OUT_MAX_ABS}) at {self.worst}, mean |d| = {mean:.3e} "
+            f"(<= {OUT_MEAN_ABS}) over {self.n} values")
+        return self.mx, mean
+
+
 def assert_lse_close(got: np.ndarray, want: np.ndarray):
     d = np.abs(got - want)
     assert float(d.max()) <= LSE_MAX_ABS, f"lse: max |d| = {float(d.max()):.3e}"

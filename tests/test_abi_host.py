@@ -248,3 +248,30 @@ def test_backward_validation_and_sizes(msa):
     assert call(**dict(kl, k_idx=P + 2)) == INVALID      # misaligned
     assert call(**dict(kl, d_idx=128)) == UNSUPPORTED
     assert call(**dict(kl, ws_bytes=need)) == WORKSPACE  # no room for the KL accumulators
+
+
+def test_static_kv2q_validation(msa):
+    """msa_build_kv2q_static validates the layout like msa_build_kv2q (every field, nb and n_windows
+    included) and rejects it on the host before touching the device."""
+    f = msa.lib.msa_build_kv2q_static
+    L = msa.msa_kv2q_layout_get(5000, 2, 128, 16)
+    assert f(None, ctypes.byref(L), P, None) == INVALID
+    assert f(P, ctypes.byref(L), None, None) == INVALID
+    assert f(P, ctypes.byref(L), P + 16, None) == INVALID       # kv2q buffer not 256-byte aligned
+    for field, delta in (("nb", 1), ("n_windows", 1), ("max_items", 1), ("total_bytes", 256), ("entries", 256)):
+        bad = msa.msa_kv2q_layout_get(5000, 2, 128, 16)
+        setattr(bad, field, getattr(bad, field) + delta)
+        assert f(P, ctypes.byref(bad), P2, None) == INVALID, field
+
+
+def test_static_kv2q_fault_injection():
+    """The host fault hook covers msa_build_kv2q_static too (fails before anything is enqueued)."""
+    code = (
+        "import sys, ctypes; sys.path.insert(0, %r)\n"
+        "import block_sparse_long_idx_b200 as m\n"
+        "L = m.msa_kv2q_layout_get(5000, 2, 128, 16)\n"
+        "r = m.lib.msa_build_kv2q_static(%d, ctypes.byref(L), %d, None)\n"
+        "print('STATUS', r)\n" % (ROOT, P, P2))
+    env = dict(os.environ, MSA_FAULT_INJECT="msa_build_kv2q_static")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert "STATUS 4" in out.stdout, out.stdout + out.stderr

@@ -63,3 +63,17 @@ def test_static_scratch_rejects_bad_layout():
     st = msa.lib.msa_build_kv2q_static(bi.data_ptr(), ctypes.byref(L), buf.data_ptr(),
                                        torch.cuda.current_stream().cuda_stream)
     assert st == 1  # MSA_ERR_INVALID_ARG
+
+
+def test_static_scratch_rejects_edited_block_count():
+    """A layout whose nb or n_windows was edited would size the kernels' counters past the kv2q
+    buffer; the entry point rejects it before enqueueing anything."""
+    bi = _selection(14)
+    H_kv, N, k = bi.shape
+    buf = torch.empty(msa.msa_kv2q_layout_get(N, H_kv, 128, k).total_bytes, dtype=torch.uint8, device="cuda")
+    for field in ("nb", "n_windows"):
+        L = msa.msa_kv2q_layout_get(N, H_kv, 128, k)
+        setattr(L, field, getattr(L, field) + 1)
+        st = msa.lib.msa_build_kv2q_static(bi.data_ptr(), ctypes.byref(L), buf.data_ptr(),
+                                           torch.cuda.current_stream().cuda_stream)
+        assert st == 1, field  # MSA_ERR_INVALID_ARG
