@@ -201,7 +201,7 @@ struct DecCfg {
     static constexpr int LD = DH + 8; // padded row (elements): conflict-free fragment loads
     // K, V, Q tiles and the per-warp max / sum; the per-warp outputs [4][16][DH] fp32 reuse the K
     // tile, which no warp reads after S (three CTAs fit per SM)
-    static constexpr int SMEM = (2 * 128 * LD + 16 * LD) * 2 + 2 * 4 * 16 * 4;
+    static constexpr int SMEM = (2 * 128 * LD + 16 * LD) * 2 + 3 * 4 * 16 * 4;
     static_assert(4 * 16 * DH * 4 <= 128 * LD * 2, "output scratch fits in the K tile");
 };
 
@@ -216,7 +216,8 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
     uint16_t* sQ = sV + 128 * LD;
     float* sO = reinterpret_cast<float*>(sK);                  // [4][16][DH], written after S
     float* sMax = reinterpret_cast<float*>(sQ + 16 * LD);     // [4][16]
-    float* sSum = sMax + 4 * 16;                               // [4][16]
+    float* sSum = sMax + 4 * 16;                               // [4][16] row sums of exp (exact)
+    float* sSumR = sSum + 4 * 16;                              // [4][16] row sums of the bf16-rounded P
 
     const int beta = blockIdx.x, r = blockIdx.y, slot = blockIdx.z;
     const int G = a.H_q / a.H_kv;
@@ -306,8 +307,10 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
     }
     const float scale = rsqrtf((float)DH);
     const float sl2 = scale * 1.4426950408889634f;
-    // P = exp(S*scale - M*scale), partial row sums, bf16 A fragments
-    float l0 = 0.f, l1 = 0.f;
+    // P = exp(S*scale - M*scale), partial row sums, bf16 A fragments. Two row sums: the exact one
+    // gives the lse (the weights the combine merges with); the sum of the bf16-rounded P the PV
+    // product uses normalises O, so each partial is an exact weighted average of V rows.
+    float l0 = 0.f, l1 = 0.f, lr0 = 0.f, lr1 = 0.f;
     uint32_t pf[2][4];
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
@@ -320,15 +323,21 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
         const int kk = n >> 1, hi = n & 1;
         pf[kk][hi * 2 + 0] = pack_bf16x2(p0, p1);
         pf[kk][hi * 2 + 1] = pack_bf16x2(p2, p3);
+        lr0 += bf16_lo(pf[kk][hi * 2 + 0]) + bf16_hi(pf[kk][hi * 2 + 0]);
+        lr1 += bf16_lo(pf[kk][hi * 2 + 1]) + bf16_hi(pf[kk][hi * 2 + 1]);
     }
 #pragma unroll
     for (int o = 1; o < 4; o <<= 1) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, o);
         l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        lr0 += __shfl_xor_sync(0xffffffffu, lr0, o);
+        lr1 += __shfl_xor_sync(0xffffffffu, lr1, o);
     }
     if (t == 0) {
         sSum[warp * 16 + g] = l0;
         sSum[warp * 16 + g + 8] = l1;
+        sSumR[warp * 16 + g] = lr0;
+        sSumR[warp * 16 + g + 8] = lr1;
     }
     // O_w = P_w V_w over this warp's 32 keys
     float oacc[DH / 8][4];
@@ -361,14 +370,15 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
     // reduce the 4 warps' partials, normalise, write the slot's partial
     for (int e = tid; e < G * DH / 2; e += 128) {
         const int row = (2 * e) / DH, col = (2 * e) % DH;
-        float o0 = 0.f, o1 = 0.f, l = 0.f;
+        float o0 = 0.f, o1 = 0.f, l = 0.f, lr = 0.f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
             o0 += sO[(w * 16 + row) * DH + col];
             o1 += sO[(w * 16 + row) * DH + col + 1];
             l += sSum[w * 16 + row];
+            lr += sSumR[w * 16 + row];
         }
-        const float inv = 1.f / l;
+        const float inv = 1.f / lr;
         const int h = r * G + row;
         // partial layout [sequence][slot][d_h/8][H_q][8] (as prefill's stage 1)
         uint32_t* dst = reinterpret_cast<uint32_t*>(a.o_part + ((int64_t)beta * a.k + slot) * a.H_q * DH +

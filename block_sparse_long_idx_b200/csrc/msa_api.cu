@@ -49,6 +49,26 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uin
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Query map of the attention's row gather. G >= 8: one box per position holds its G heads x d_h
+// columns: a 5-D view of q[N][H_q][d_h] with dims (64 columns, 8 heads, 64-column chunk, head group
+// of 8, position), so the box lands in shared memory as [head group][chunk][8 heads][128 B] and the
+// tile's 8-row groups are a uniform 1024 * d_h / 64 bytes apart. G < 8: one 3-D box of G heads x 64
+// columns per 64-column chunk.
+bool make_qmap(CUtensorMap* m, const void* q, int d_h, int H_q, int64_t N, int G)
+{
+    if (G < 8) return make_map_3d(m, q, d_h, H_q, N, 64, G, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t nkc = (cuuint64_t)d_h / 64;
+    const cuuint64_t dims[5] = {64, 8, nkc, (cuuint64_t)H_q / 8, (cuuint64_t)N};
+    const cuuint64_t strides[4] = {(cuuint64_t)d_h * 2, 128, (cuuint64_t)8 * d_h * 2, (cuuint64_t)H_q * d_h * 2};
+    const cuuint32_t box[5] = {64, 8, (cuuint32_t)nkc, (cuuint32_t)(G / 8), 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(q), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -456,7 +476,7 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
     float* lse_part = (float*)(ws + used + align_up((size_t)rows_pass * k * H_q * d_h * 2, 256));
 
     CUtensorMap qmap, kmap, vmap;
-    if (!make_map_3d(&qmap, q, d_h, H_q, N, 64, G, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_qmap(&qmap, q, d_h, H_q, N, G) ||
         !make_map_3d(&kmap, kk, d_h, H_kv, N, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_3d(&vmap, v, d_h, H_kv, N, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B))
         return MSA_ERR_INVALID_ARG;
@@ -749,7 +769,7 @@ msa_status msa_sparse_prefill_varlen(const msa_bf16* q, const msa_bf16* kk, cons
     const CUtensorMapSwizzle sw = d_idx == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     if (!make_map_3d(&qim, q_idx, d_idx, H_kv, T, box0, 1, kBk, sw) ||
         !make_map_3d(&kim, k_idx, d_idx, H_kv, Tk, box0, 1, kBk, sw) ||
-        !make_map_3d(&qmap, q, d_h, H_q, T, 64, G, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_qmap(&qmap, q, d_h, H_q, T, G) ||
         !make_map_3d(&kmap, kk, d_h, H_kv, Tk, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_3d(&vmap, v, d_h, H_kv, Tk, 64, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B))
         return MSA_ERR_INVALID_ARG;

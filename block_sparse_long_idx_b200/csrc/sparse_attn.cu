@@ -4,19 +4,19 @@
 // Each work item is one (group r, KV block b, chunk of the rows that selected b). Its K and V blocks
 // are staged in shared memory once by TMA; the rows are processed in 128-row tensor-core tiles made
 // of 128/G query positions x G heads ("query concatenation"), each position's G heads gathered by
-// one TMA box from q[p, r*G .. r*G+G, :]. Per tile:
+// TMA from q[p, r*G .. r*G+G, :] (one box per position when G >= 8). Per tile:
 //   S = Q K^T                         tcgen05.mma, A = Q (smem), B = K (smem), D in TMEM
 //   P = exp(S*scale - rowmax)         softmax warps, thread = TMEM lane = tile row; the causal mask
 //                                     only applies to rows whose own block is b; P goes back to
 //                                     TMEM as bf16 over the first 64 S columns
+//   partial[p, slot, h] = O / rowsum(bf16 P), lse = rowmax*scale + log(rowsum(P))
 //   O = P V                           tcgen05.mma, A = P (TMEM), B = V (smem, MN-major)
-//   partial[p, slot, h] = O / rowsum, lse = rowmax*scale + log(rowsum)
 // A work item covers one KV block only, so no running-max rescaling is needed. Stage 2
 // (combine.cu) merges the <= k partials of every (row, head) through their lse.
 //
 // Roles (512 threads, four warpgroups):
 //   WG0: warp 0 = K/V TMA producer, warp 1 = S issuer + TMEM owner, warp 2 = tile scheduler and Q
-//        gather (one TMA box per position, issued by the 32 lanes in parallel), warp 3 = PV issuer
+//        gather (TMA boxes issued by the 32 lanes in parallel), warp 3 = PV issuer
 //   WG1, WG2: softmax of even / odd tiles
 //   WG3: epilogue of every tile (O / rowsum -> partial slot)
 // Work items are claimed dynamically: the tile scheduler takes the next item of the launch's work
@@ -28,15 +28,22 @@
 // waits on a global load. The epilogue releases a record after its tile's PV. For a packed batch
 // of sequences the block tables give each global block's first key row (K/V coordinates) and the
 // query-row coordinate of its first token (the causal mask on the diagonal block).
-// TMEM (512 columns): two 128-column S/P regions A[t % 2] at columns 0 and 128 (S, then P in
-// columns 0-63) and two output regions O[t % 2] at columns 256 and 384. Two threads issue the
-// MMAs, so neither's polling leaves the tensor pipe idle: the S issuer issues S(t) once PV(t-2)
-// has consumed P(t-2) (region A[t % 2] free); the PV issuer issues PV(t) once P(t) is written and
-// the epilogue of t-2 has read O[t % 2], which leaves the epilogue a full tile of slack.
-// Barriers: s_full[2], p_full[2], pv_done[2] per S/P region; o_full[2], o_free[2] per O region;
-// ml_full[4] hands each tile's row max and row sum from the softmax to the epilogue through shared
-// memory (slot t % 4, rewritten by the softmax of t+4, which needs S(t+4), which needs PV(t+2),
-// which needs the epilogue of t to have read O).
+//
+// Pipeline depth. A tile's S/P columns stay busy from S through the softmax until PV has read P,
+// while its output columns are busy only from PV until the epilogue has read them, so TMEM (512
+// columns) holds three S/P regions R[t % 3] at columns 0, 128, 256 (S, then P in the first 64
+// columns) and one output region at columns 384-511: three tiles are in flight between S and PV.
+// Two threads issue the MMAs: the S issuer issues S(t) once PV(t-3) has consumed P(t-3) (region
+// R[t % 3] free) and Q(t) has landed; the PV issuer issues PV(t) once P(t) is written and the
+// epilogue has read O(t-1). Q has three shared-memory stages (stage t % 3, refilled for t+3 once
+// S(t) has completed). K and V of consecutive items rotate through three 128-row buffers in load
+// order K0 V0 K1 V1 ...: load n goes to buffer n % 3 once load n-3 is released (the K of an item
+// after its last S, its V after its last PV), so the next item's K and V stream in while the
+// current item's tiles run.
+// Barriers: s_full, p_full, pv_done per S/P region; o_full, o_free for the output region; ml_full[4]
+// hands each tile's lse and 1 / (rounded row sum) from the softmax to the epilogue through shared memory
+// (slot t % 4, rewritten by the softmax of t+4, which needs S(t+4), which needs PV(t+1), which needs
+// the epilogue of t to have read O(t), after it read the slot).
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -46,34 +53,47 @@ namespace msa {
 
 namespace {
 
-template <int DH>
+template <int DH, int G>
 struct AttnCfg {
     static constexpr int NKC = DH / 64;          // 64-column (128-byte) chunks
     static constexpr int CHUNK = 128 * 128;      // bytes per chunk of a 128-row tile
     static constexpr int TILE = NKC * CHUNK;     // Q, K or V tile bytes
-    static constexpr int NQ = 2;                 // Q stages
-    static constexpr int SMEM = 1024 + NQ * TILE + 4 * TILE;
+    static constexpr int NQ = 3;                 // Q stages
+    static constexpr int NKV = 3;                // K/V buffers
+    static constexpr int SMEM = 1024 + (NQ + NKV) * TILE;
+    // Q tile layout. G >= 8: position-major, one TMA box per position laid out as
+    // [head group of 8][chunk][8 heads][128 B]: 8-row group g = p * G/8 + hg sits at g * QSBO and
+    // chunk c at + c * 1024. G < 8: chunk-major like K ([chunk][row][128 B]), one box per
+    // (position, chunk).
+    static constexpr bool QPOS = G >= 8;
+    static constexpr int QSBO = QPOS ? NKC * 1024 : 1024; // bytes between 8-row groups
+    static constexpr int QCHUNK = QPOS ? 1024 : CHUNK;    // bytes between 64-column chunks
 };
 
-constexpr int kRing = 8; // tile records in flight between the scheduler and the epilogue
+constexpr int kRing = 8;    // tile records in flight between the scheduler and the epilogue
+constexpr int kRegions = 3; // S/P regions in TMEM
+constexpr uint32_t kOCol = 384;
 
 struct TileRec {
     int32_t r, b;  // GQA group, KV block
     int32_t npos;  // positions in the tile (1 .. 128/G); -1 marks the end of the CTA's work
-    int32_t flags; // bit 0: first tile of its item, bit 1: last tile, bit 2: K/V stage of the item
+    int32_t flags; // bit 0: first tile of its item, bit 1: last tile
     int32_t tok0;  // query-row coordinate of block b's first token (b * 128 for one sequence)
 };
 
 struct AttnShared {
-    uint64_t kv_full[2], kv_empty[2];
-    uint64_t q_full[2], q_empty[2];
-    uint64_t s_full[2], p_full[2], pv_done[2];
-    uint64_t o_full[2], o_free[2];
+    uint64_t kv_full[3], kv_empty[3];
+    uint64_t q_full[3], q_empty[3];
+    uint64_t s_full[kRegions], p_full[kRegions], pv_done[kRegions];
+    uint64_t o_full, o_free;
     uint64_t ml_full[4];
     uint64_t tile_full[kRing], tile_free[kRing];
     uint64_t kvrec_full[4], kvrec_free[4];
-    uint64_t done, done2;
-    float2 ml[4][128]; // (row max of the raw scores, row sum of exp) per tile slot and row
+    uint64_t done;
+    uint64_t xbar[2][4];    // [tile & 1][lane quarter]: both softmax warps of the quarter hold their max
+    float xmax[2][2][128];  // [tile & 1][column half][row]: the halves' row maxima, exchanged
+    float mrow[4][128];     // [tile slot][row]: row max of the raw scores
+    float2 lsum[4][2][128]; // [tile slot][column half][row]: (sum of exp, sum of the bf16-rounded P)
     TileRec rec[kRing];
     msa_work_item kvrec[4]; // items handed to the K/V producer (len = 0: no more work)
     int32_t rec_e[kRing][128]; // entry (i*k + slot) of each position of the tile
@@ -83,26 +103,24 @@ struct AttnShared {
 
 constexpr uint32_t kNegInfBits = 0xff800000u;
 constexpr int REG_LAUNCH = 128; // 65536 registers / 512 threads
-constexpr int REG_PRODUCER = 56, REG_SOFTMAX = 184, REG_EPILOGUE = 88;
+constexpr int REG_PRODUCER = 96, REG_SOFTMAX = 128, REG_EPILOGUE = 160;
 static_assert(REG_PRODUCER + 2 * REG_SOFTMAX + REG_EPILOGUE <= 4 * REG_LAUNCH, "register split exceeds the launch budget");
 
-__device__ __forceinline__ uint32_t a_col(int t) { return (uint32_t)(t & 1) * 128; }
-__device__ __forceinline__ uint32_t o_col(int t) { return 256u + (uint32_t)(t & 1) * 128; }
+__device__ __forceinline__ uint32_t a_col(int t) { return (uint32_t)(t % kRegions) * 128; }
 
 template <int DH, int G>
 __global__ void __launch_bounds__(512, 1)
     sparse_attn_kernel(AttnArgs a, const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap)
 {
-    using C = AttnCfg<DH>;
+    using C = AttnCfg<DH, G>;
     constexpr int PPT = 128 / G;
-    constexpr int NQ = C::NQ;
+    constexpr int NQ = C::NQ, NKV = C::NKV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;                  // [NQ][TILE]
-    uint8_t* sK = smem + NQ * C::TILE;   // [2][TILE]
-    uint8_t* sV = sK + 2 * C::TILE;      // [2][TILE]
-    AttnShared& sh = *reinterpret_cast<AttnShared*>(sV + 2 * C::TILE);
+    uint8_t* sKV = smem + NQ * C::TILE;  // [NKV][TILE]
+    AttnShared& sh = *reinterpret_cast<AttnShared*>(sKV + NKV * C::TILE);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wg = warp >> 2;
@@ -114,26 +132,27 @@ __global__ void __launch_bounds__(512, 1)
     const bool tl_on = a.timeline != nullptr && cta == 0;
 #define TL(slot, tile)                                                                                    \
     do {                                                                                                  \
-        if (tl_on && (tile) < a.timeline_tiles) a.timeline[(int64_t)(tile) * 16 + (slot)] = clock64();    \
+        if (tl_on && (tile) < a.timeline_tiles) a.timeline[(int64_t)(tile) * 32 + (slot)] = clock64();    \
     } while (0)
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NKV; ++i) {
             mbar_init(&sh.kv_full[i], 1);
             mbar_init(&sh.kv_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kRegions; ++i) {
             mbar_init(&sh.s_full[i], 1);
-            mbar_init(&sh.p_full[i], 4);
+            mbar_init(&sh.p_full[i], 8);
             mbar_init(&sh.pv_done[i], 1);
-            mbar_init(&sh.o_full[i], 1);
-            mbar_init(&sh.o_free[i], 4);
         }
+        mbar_init(&sh.o_full, 1);
+        mbar_init(&sh.o_free, 4);
         for (int i = 0; i < NQ; ++i) {
             mbar_init(&sh.q_full[i], 1);
             mbar_init(&sh.q_empty[i], 1);
         }
-        for (int i = 0; i < 4; ++i) mbar_init(&sh.ml_full[i], 4);
+        for (int i = 0; i < 4; ++i) mbar_init(&sh.ml_full[i], 8);
+        for (int i = 0; i < 8; ++i) mbar_init(&sh.xbar[i >> 2][i & 3], 2);
         for (int i = 0; i < kRing; ++i) {
             mbar_init(&sh.tile_full[i], 1);
             mbar_init(&sh.tile_free[i], 4);
@@ -143,7 +162,6 @@ __global__ void __launch_bounds__(512, 1)
             mbar_init(&sh.kvrec_free[i], 1);
         }
         mbar_init(&sh.done, 1);
-        mbar_init(&sh.done2, 1);
         sh.abort_flag = 0;
         fence_mbar_init();
     }
@@ -160,26 +178,32 @@ __global__ void __launch_bounds__(512, 1)
         reg_set<REG_PRODUCER, REG_LAUNCH>();
         if (warp == 0) {
             // -------------------------------------------------------- K/V producer
+            // loads n = 2i (K of item i) and 2i+1 (V of item i) go to buffer n % 3
             if (lane == 0) {
-                int it = 0;
-                for (;; ++it) {
+                int n = 0;
+                bool ok = true;
+                for (int it = 0; ok; ++it) {
                     const int s4 = it & 3;
                     if (!wait_or_abort(&sh.kvrec_full[s4], (it >> 2) & 1, abort_flag, a.err, 38, kWaitLimit)) break;
                     const msa_work_item item = sh.kvrec[s4];
                     mbar_arrive(&sh.kvrec_free[s4]);
                     if (item.len <= 0) break;
-                    const int s = it & 1;
-                    if (!wait_or_abort(&sh.kv_empty[s], ((it >> 1) & 1) ^ 1, abort_flag, a.err, 20, kWaitLimit))
-                        break;
                     const int tok0 = a.blk_tok ? a.blk_tok[item.b] : item.b * kBk;
-                    mbar_arrive_expect_tx(&sh.kv_full[s], 2 * C::TILE);
-                    for (int c = 0; c < C::NKC; ++c) {
-                        tma_load_3d(sK + s * C::TILE + c * C::CHUNK, &kmap, &sh.kv_full[s], c * 64, item.r, tok0);
-                        tma_load_3d(sV + s * C::TILE + c * C::CHUNK, &vmap, &sh.kv_full[s], c * 64, item.r, tok0);
+                    for (int kv = 0; kv < 2; ++kv, ++n) {
+                        const int buf = n % NKV;
+                        if (!wait_or_abort(&sh.kv_empty[buf], ((n / NKV) & 1) ^ 1, abort_flag, a.err, 20,
+                                           kWaitLimit)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&sh.kv_full[buf], C::TILE);
+                        for (int c = 0; c < C::NKC; ++c)
+                            tma_load_3d(sKV + buf * C::TILE + c * C::CHUNK, kv ? &vmap : &kmap, &sh.kv_full[buf],
+                                        c * 64, item.r, tok0);
                     }
                 }
-                for (int g = it - 1; g >= 0 && g >= it - 2; --g)
-                    drain_wait(&sh.kv_full[g & 1], (g >> 1) & 1, a.err, 40, kWaitLimit);
+                for (int g = n - 1; g >= 0 && g >= n - NKV; --g)
+                    drain_wait(&sh.kv_full[g % NKV], (g / NKV) & 1, a.err, 40, kWaitLimit);
             }
         } else if (warp == 2) {
             // -------------------------------------------------------- tile scheduler + Q gather
@@ -242,8 +266,7 @@ __global__ void __launch_bounds__(512, 1)
                         if (pl < npos) sh.rec_e[rs][pl] = e[u];
                     }
                     if (lane == 0)
-                        sh.rec[rs] = TileRec{item.r, item.b, npos,
-                                             (t == 0 ? 1 : 0) | (t == ntiles - 1 ? 2 : 0) | ((it & 1) << 2), tok0};
+                        sh.rec[rs] = TileRec{item.r, item.b, npos, (t == 0 ? 1 : 0) | (t == ntiles - 1 ? 2 : 0), tok0};
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh.tile_full[rs]);
                     if (lane == 0)
@@ -262,10 +285,16 @@ __global__ void __launch_bounds__(512, 1)
                     for (int u = 0; u < (PPT + 31) / 32; ++u) {
                         const int pl = lane + 32 * u;
                         if (pl < npos) {
+                            uint8_t* dst = sQ + qs * C::TILE;
+                            if constexpr (C::QPOS) {
+                                tma_load_5d(dst + pl * (G * DH * 2), &qmap, &sh.q_full[qs], 0, 0, 0, item.r * (G / 8),
+                                            e[u] / a.k);
+                            } else {
 #pragma unroll
-                            for (int c = 0; c < C::NKC; ++c)
-                                tma_load_3d(sQ + qs * C::TILE + c * C::CHUNK + pl * G * 128, &qmap, &sh.q_full[qs],
-                                            c * 64, item.r * G, e[u] / a.k);
+                                for (int c = 0; c < C::NKC; ++c)
+                                    tma_load_3d(dst + c * C::CHUNK + pl * G * 128, &qmap, &sh.q_full[qs], c * 64,
+                                                item.r * G, e[u] / a.k);
+                            }
                         }
                     }
                     if (lane == 0) TL(1, qt);
@@ -274,13 +303,11 @@ __global__ void __launch_bounds__(512, 1)
                 ++it;
             }
             const int n_tiles = qt;
-            // two end records, so that each softmax warpgroup (even / odd tiles) meets one
+            // the end record, read by every consumer role
             if (lane == 0 && ok) {
-                for (int z = 0; z < 2; ++z, ++qt) {
-                    const int rs = qt % kRing;
-                    if (qt >= kRing && !wait_or_abort(&sh.tile_free[rs], ((qt / kRing) & 1) ^ 1, abort_flag, a.err,
-                                                      33, kWaitLimit))
-                        break;
+                const int rs = qt % kRing;
+                if (qt < kRing ||
+                    wait_or_abort(&sh.tile_free[rs], ((qt / kRing) & 1) ^ 1, abort_flag, a.err, 33, kWaitLimit)) {
                     sh.rec[rs] = TileRec{0, 0, -1, 0, 0};
                     mbar_arrive(&sh.tile_full[rs]);
                 }
@@ -289,130 +316,185 @@ __global__ void __launch_bounds__(512, 1)
                 for (int g = n_tiles - 1; g >= 0 && g >= n_tiles - NQ; --g)
                     drain_wait(&sh.q_full[g % NQ], (g / NQ) & 1, a.err, 41, kWaitLimit);
         } else if (warp == 1) {
-            // -------------------------------------------------------- S issuer: S(t) = Q K^T
+            // -------------------------------------------------------- MMA issuer (S and PV)
+            // One thread issues every MMA. A ready PV goes first: it gates the epilogue, the output
+            // region and the S/P region of the tile three ahead, while an S issued early only waits
+            // in the tensor pipe. S(ts) needs its record, Q(ts), the item's K and PV(ts-3) complete;
+            // PV(tp) needs S(tp) issued, P(tp), the item's V and the epilogue's read of O(tp-1).
             if (lane == 0) {
                 constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
-                const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
-                int it = -1;
-                uint64_t kdesc = 0;
-                for (int qt = 0;; ++qt) {
-                    const int rs = qt % kRing;
-                    if (!poll_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 34, kWaitLimit)) break;
-                    const TileRec rec = sh.rec[rs];
-                    if (rec.npos < 0) break;
-                    const int kvs = (rec.flags >> 2) & 1;
-                    if (rec.flags & 1) {
-                        ++it;
-                        if (!poll_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 23, kWaitLimit)) break;
-                        TL(8, qt);
-                        kdesc = desc_kmajor(aK + kvs * C::TILE, 128);
-                    }
-                    const int qa = qt & 1, qs = qt % NQ;
-                    // A[qt % 2] is free once PV(qt-2) has consumed P(qt-2)
-                    if (!poll_or_abort(&sh.q_full[qs], (qt / NQ) & 1, abort_flag, a.err, 24, kWaitLimit) ||
-                        (qt >= 2 && !poll_or_abort(&sh.pv_done[qa], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 25,
-                                                   kWaitLimit)))
-                        break;
-                    TL(9, qt);
-                    tc_fence_after();
-                    const uint64_t qdesc = desc_kmajor(aQ + qs * C::TILE, 128);
-                    const uint32_t sd = tmem + a_col(qt);
+                constexpr uint32_t idPV = idesc_bf16_f32(128, DH, true);
+                const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV);
+                int ts = 0, tp = 0;     // next tile for S, for PV
+                int its = -1, itp = -1; // item counters of the two sides
+                int kb = 0, vb = 0;
+                bool s_rec = false, p_rec = false, s_end = false, p_end = false;
+                bool s_kv = false, p_kv = false; // the K (V) of the pending tile's item has landed
+                bool p_pf = false, p_of = false; // P(tp) written, O(tp-1) read
+                bool s_q = false, s_pv = false;  // Q(ts) landed, PV(ts-3) complete
+                TileRec rs_{}, rp_{};
+                uint64_t kdesc = 0, vdesc = 0;
+                long long t_last = clock64();
+                while (!(s_end && p_end)) {
+                    bool progress = false;
+                    // ---------------- PV(tp)
+                    if (!p_end && tp < ts) {
+                        if (!p_rec && mbar_poll(&sh.tile_full[tp % kRing], (tp / kRing) & 1)) {
+                            rp_ = sh.rec[tp % kRing];
+                            p_rec = true;
+                            if (rp_.flags & 1) {
+                                ++itp;
+                                vb = (2 * itp + 1) % NKV;
+                                p_kv = false;
+                            }
+                        }
+                        if (p_rec && !p_kv && mbar_poll(&sh.kv_full[vb], ((2 * itp + 1) / NKV) & 1)) {
+                            p_kv = true;
+                            vdesc = smem_desc(aKV + vb * C::TILE, C::CHUNK, 1024, 128);
+                        }
+                        const int reg = tp % kRegions;
+                        if (p_rec && !p_pf && mbar_poll(&sh.p_full[reg], (tp / kRegions) & 1)) {
+                            p_pf = true;
+                            TL(10, tp);
+                        }
+                        if (p_rec && !p_of && mbar_poll(&sh.o_free, (tp & 1) ^ 1)) {
+                            p_of = true;
+                            TL(11, tp);
+                        }
+                        if (p_rec && p_kv && p_pf && p_of) {
+                            TL(12, tp);
+                            tc_fence_after();
+                            const uint32_t acol = tmem + a_col(tp);
 #pragma unroll
-                    for (int ks = 0; ks < DH / 16; ++ks) {
-                        const uint64_t off = (uint64_t)((((ks >> 2) * C::CHUNK) + (ks & 3) * 32) >> 4);
-                        mma_ss(sd, qdesc + off, kdesc + off, idS, ks > 0);
+                            for (int ks = 0; ks < 8; ++ks) // 16 keys = 2048 bytes of V per step
+                                mma_ts(tmem + kOCol, acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
+                            tc_commit(&sh.pv_done[reg]);
+                            tc_commit(&sh.o_full);
+                            if (rp_.flags & 2) tc_commit(&sh.kv_empty[vb]); // the item's V is no longer read
+                            TL(3, tp);
+                            ++tp;
+                            p_rec = p_pf = p_of = false;
+                            progress = true;
+                        }
+                    } else if (!p_end && s_end && tp == ts) {
+                        p_end = true; // every issued S has its PV
                     }
-                    tc_commit(&sh.s_full[qa]);
-                    tc_commit(&sh.q_empty[qs]);
-                    TL(2, qt);
+                    // ---------------- S(ts)
+                    if (!s_end) {
+                        if (!s_rec && mbar_poll(&sh.tile_full[ts % kRing], (ts / kRing) & 1)) {
+                            rs_ = sh.rec[ts % kRing];
+                            s_rec = true;
+                            if (rs_.npos < 0) {
+                                s_end = true;
+                            } else if (rs_.flags & 1) {
+                                ++its;
+                                kb = (2 * its) % NKV;
+                                s_kv = false;
+                            }
+                        }
+                        if (s_rec && !s_end && !s_kv && mbar_poll(&sh.kv_full[kb], ((2 * its) / NKV) & 1)) {
+                            s_kv = true;
+                            kdesc = desc_kmajor(aKV + kb * C::TILE, 128);
+                            TL(8, ts);
+                        }
+                        const int reg = ts % kRegions, qs = ts % NQ;
+                        // region R[ts % 3] is free once PV(ts-3) has consumed P(ts-3)
+                        if (s_rec && !s_end && !s_q && mbar_poll(&sh.q_full[qs], (ts / NQ) & 1)) s_q = true;
+                        if (s_rec && !s_end && !s_pv && mbar_poll(&sh.pv_done[reg], ((ts / kRegions) & 1) ^ 1))
+                            s_pv = true;
+                        if (s_rec && !s_end && s_kv && s_q && s_pv) {
+                            TL(9, ts);
+                            tc_fence_after();
+                            const uint64_t qdesc = smem_desc(aQ + qs * C::TILE, 16, C::QSBO, 128);
+                            const uint32_t sd = tmem + a_col(ts);
+#pragma unroll
+                            for (int ks = 0; ks < DH / 16; ++ks) {
+                                const uint64_t qoff = (uint64_t)((((ks >> 2) * C::QCHUNK) + (ks & 3) * 32) >> 4);
+                                const uint64_t koff = (uint64_t)((((ks >> 2) * C::CHUNK) + (ks & 3) * 32) >> 4);
+                                mma_ss(sd, qdesc + qoff, kdesc + koff, idS, ks > 0);
+                            }
+                            tc_commit(&sh.s_full[reg]);
+                            tc_commit(&sh.q_empty[qs]);
+                            if (rs_.flags & 2) tc_commit(&sh.kv_empty[kb]); // the item's K is no longer read
+                            TL(2, ts);
+                            ++ts;
+                            s_rec = s_q = s_pv = false;
+                            progress = true;
+                        }
+                    }
+                    if (progress) {
+                        t_last = clock64();
+                    } else {
+                        // back off briefly: a spinning thread takes issue slots from the softmax and
+                        // epilogue warps of its SM sub-partition, which produce the next events
+                        __nanosleep(32);
+                        if (*abort_flag) break;
+                        if (clock64() - t_last > kWaitLimit) {
+                            report_error(a.err, MSA_ERR_TIMEOUT, 25);
+                            *abort_flag = 1;
+                            break;
+                        }
+                    }
                 }
                 tc_commit(&sh.done);
                 drain_wait(&sh.done, 0, a.err, 42, kWaitLimit);
-            }
-        } else if (warp == 3) {
-            // -------------------------------------------------------- PV issuer: O(t) = P(t) V
-            if (lane == 0) {
-                constexpr uint32_t idPV = idesc_bf16_f32(128, DH, true);
-                const uint32_t aV = smem_u32(sV);
-                int it = -1;
-                uint64_t vdesc = 0;
-                for (int qt = 0;; ++qt) {
-                    const int rs = qt % kRing;
-                    if (!poll_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 35, kWaitLimit)) break;
-                    const TileRec rec = sh.rec[rs];
-                    if (rec.npos < 0) break;
-                    const int kvs = (rec.flags >> 2) & 1;
-                    if (rec.flags & 1) {
-                        ++it;
-                        if (!poll_or_abort(&sh.kv_full[kvs], (it >> 1) & 1, abort_flag, a.err, 30, kWaitLimit)) break;
-                        vdesc = smem_desc(aV + kvs * C::TILE, C::CHUNK, 1024, 128);
-                    }
-                    const int pa = qt & 1;
-                    TL(10, qt);
-                    // needs P(qt) and the epilogue of qt-2 to have read O[qt % 2]
-                    if (!poll_or_abort(&sh.p_full[pa], (qt >> 1) & 1, abort_flag, a.err, 22, kWaitLimit) ||
-                        (qt >= 2 && !poll_or_abort(&sh.o_free[pa], ((qt >> 1) & 1) ^ 1, abort_flag, a.err, 28,
-                                                   kWaitLimit)))
-                        break;
-                    TL(12, qt);
-                    tc_fence_after();
-                    const uint32_t acol = tmem + a_col(qt);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) // 16 keys = 2048 bytes of V per step
-                        mma_ts(tmem + o_col(qt), acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
-                    tc_commit(&sh.pv_done[pa]);
-                    tc_commit(&sh.o_full[pa]);
-                    if (rec.flags & 2) tc_commit(&sh.kv_empty[kvs]);
-                    TL(3, qt);
-                }
-                tc_commit(&sh.done2);
-                drain_wait(&sh.done2, 0, a.err, 43, kWaitLimit);
             }
         }
     } else if (wg <= 2) {
         reg_set<REG_SOFTMAX, REG_LAUNCH>();
         // ------------------------------------------------------------ softmax
+        // Both warpgroups work on every tile: warpgroup beta takes key columns 64*beta .. +63 of the
+        // rows of its TMEM lane quarter. The two warps of a lane quarter exchange their row maxima
+        // through shared memory (an mbarrier per tile parity and quarter, two arrivals), then each
+        // writes its half of P.
         const int beta = wg - 1;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int pl = row / G;
         const float sl2 = rsqrtf((float)DH) * 1.4426950408889634f;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        for (int qt = beta;; qt += 2) {
+        for (int qt = 0;; ++qt) {
             const int rs = qt % kRing;
             if (!wait_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 36, kWaitLimit)) break;
             const TileRec rec = sh.rec[rs];
             if (rec.npos < 0) break;
-            const int qa = qt & 1;
-            const int limit = pl < rec.npos ? min(127, sh.rec_e[rs][pl] / a.k - rec.tok0) : 127;
-            if (!wait_or_abort(&sh.s_full[qa], (qt >> 1) & 1, abort_flag, a.err, 26, kWaitLimit)) break;
-            if (row == 0) TL(4, qt);
+            const int reg = qt % kRegions;
+            // last visible key column of this half (keys after the query are masked on the diagonal block)
+            const int limit =
+                (pl < rec.npos ? min(127, sh.rec_e[rs][pl] / a.k - rec.tok0) : 127) - 64 * beta;
+            if (!wait_or_abort(&sh.s_full[reg], (qt / kRegions) & 1, abort_flag, a.err, 26, kWaitLimit)) break;
+            if (row == 0 && beta == 0) TL(4, qt);
             tc_fence_after();
             const uint32_t sadr = lane_base + a_col(qt);
-            uint32_t s[128];
-            tmem_ld32_at<0>(sadr, s);
-            tmem_ld32_at<32>(sadr + 32, s);
-            tmem_ld32_at<64>(sadr + 64, s);
-            tmem_ld32_at<96>(sadr + 96, s);
+            uint32_t s[64];
+            tmem_ld32_at<0>(sadr + 64 * beta, s);
+            tmem_ld32_at<32>(sadr + 64 * beta + 32, s);
             tmem_ld_wait();
-            if (row == 0) TL(14, qt);
-            if (limit < 127) { // the query's own block: keys after the query are invisible
+            if (row == 0 && beta == 0) TL(14, qt);
+            if (limit < 63) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
+                for (int c = 0; c < 64; ++c)
                     if (c > limit) s[c] = kNegInfBits;
             }
             float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F;
 #pragma unroll
-            for (int c = 0; c < 128; c += 4) {
+            for (int c = 0; c < 64; c += 4) {
                 m0 = max3f(m0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
                 m1 = max3f(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
             }
-            const float m = fmaxf(m0, m1);
+            sh.xmax[qt & 1][beta][row] = fmaxf(m0, m1);
+            // both halves of S are in registers before either half's P overwrites TMEM columns 0-63
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.xbar[qt & 1][quarter]);
+            if (!wait_or_abort(&sh.xbar[qt & 1][quarter], (qt >> 1) & 1, abort_flag, a.err, 44, kWaitLimit)) break;
+            tc_fence_after();
+            const float m = fmaxf(sh.xmax[qt & 1][0][row], sh.xmax[qt & 1][1][row]);
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t nmx2 = f2_pack(-m * sl2, -m * sl2);
-            uint64_t l2 = 0;
+            uint64_t l2 = 0, lr2 = 0;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
@@ -420,20 +502,25 @@ __global__ void __launch_bounds__(512, 1)
                     const uint64_t xx = f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2x2,
                                                nmx2);
                     const float e0 = ex2_approx(f2_lo(xx)), e1 = ex2_approx(f2_hi(xx));
-                    l2 = f2_add(l2, f2_pack(e0, e1));
                     pk[q] = pack_bf16x2(e0, e1);
+                    l2 = f2_add(l2, f2_pack(e0, e1));
+                    lr2 = f2_add(lr2, f2_pack(bf16_lo(pk[q]), bf16_hi(pk[q])));
                 }
-                tmem_st16(sadr + c4 * 16, pk);
+                tmem_st16(sadr + 32 * beta + c4 * 16, pk);
             }
-            sh.ml[qt & 3][row] = make_float2(m, f2_lo(l2) + f2_hi(l2));
+            // the exact sum gives the lse (the combine's merge weight); the sum of the bf16-rounded P
+            // that the PV product uses normalises O, so each partial is an exact weighted average
+            sh.lsum[qt & 3][beta][row] = make_float2(f2_lo(l2) + f2_hi(l2), f2_lo(lr2) + f2_hi(lr2));
+            if (beta == 0) sh.mrow[qt & 3][row] = m;
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&sh.p_full[qa]);
+                mbar_arrive(&sh.p_full[reg]);
                 mbar_arrive(&sh.ml_full[qt & 3]);
+                TL(16 + 4 * beta + quarter, qt);
             }
-            if (row == 0) TL(5, qt);
+            if (row == 0 && beta == 0) TL(5, qt);
         }
     } else {
         reg_set<REG_EPILOGUE, REG_LAUNCH>();
@@ -453,13 +540,14 @@ __global__ void __launch_bounds__(512, 1)
             const int32_t e = valid ? sh.rec_e[rs][pl] : 0;
             const int p = e / a.k;
             const int slot = e - p * a.k;
-            if (!wait_or_abort(&sh.o_full[qt & 1], (qt >> 1) & 1, abort_flag, a.err, 27, kWaitLimit) ||
+            if (!wait_or_abort(&sh.o_full, qt & 1, abort_flag, a.err, 27, kWaitLimit) ||
                 !wait_or_abort(&sh.ml_full[qt & 3], (qt >> 2) & 1, abort_flag, a.err, 29, kWaitLimit))
                 break;
             if (row == 0) TL(6, qt);
             tc_fence_after();
-            const float2 ml = sh.ml[qt & 3][row];
-            const float inv_l = 1.f / ml.y;
+            const float2 la = sh.lsum[qt & 3][0][row], lb = sh.lsum[qt & 3][1][row];
+            const float lse_row = sh.mrow[qt & 3][row] * scale + logf(la.x + lb.x);
+            const float inv_l = 1.f / (la.y + lb.y);
             const int h = rec.r * G + hh;
             const int64_t prow = (int64_t)(p - a.row0);
             bool store = valid;
@@ -471,36 +559,37 @@ __global__ void __launch_bounds__(512, 1)
             // 16-byte units, so each warp-wide store writes contiguous runs
             uint4* d4 = reinterpret_cast<uint4*>(a.o_part + (prow * a.k + slot) * (int64_t)a.H_q * DH) + h;
             const uint64_t il2 = f2_pack(inv_l, inv_l);
+            // the whole output row is read (64-column halves, converted to bf16 as they arrive) before
+            // any store, and the region is released to the next PV right after the last read
+            uint32_t w[DH / 2];
 #pragma unroll
-            for (int c = 0; c < DH / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + o_col(qt) + c * 32, o);
+            for (int hf = 0; hf < DH / 64; ++hf) {
+                uint32_t o[64];
+                tmem_ld32_at<0>(lane_base + kOCol + hf * 64, o);
+                tmem_ld32_at<32>(lane_base + kOCol + hf * 64 + 32, o);
                 tmem_ld_wait();
-                if (c == DH / 32 - 1) { // O fully read: PV of the next tile may overwrite it
+                if (hf == DH / 64 - 1) { // O fully read: the next tile's PV may overwrite it
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive(&sh.o_free[qt & 1]);
+                        mbar_arrive(&sh.o_free);
                         mbar_arrive(&sh.tile_free[rs]); // S, softmax and PV of qt are done with the record
+                        TL(24 + quarter, qt);
                     }
                     if (row == 0) TL(13, qt);
                 }
-                if (store) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int z = 0; z < 4; ++z) {
-                            const uint64_t y = f2_mul(
-                                f2_pack(__uint_as_float(o[8 * q + 2 * z]), __uint_as_float(o[8 * q + 2 * z + 1])),
-                                il2);
-                            w[z] = pack_bf16x2(f2_lo(y), f2_hi(y));
-                        }
-                        d4[(c * 4 + q) * a.H_q] = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
+                for (int z = 0; z < 32; ++z) {
+                    const uint64_t y = f2_mul(f2_pack(__uint_as_float(o[2 * z]), __uint_as_float(o[2 * z + 1])), il2);
+                    w[hf * 32 + z] = pack_bf16x2(f2_lo(y), f2_hi(y));
                 }
             }
-            if (store) a.lse_part[(prow * a.k + slot) * a.H_q + h] = ml.x * scale + logf(ml.y);
+            if (store) {
+#pragma unroll
+                for (int u = 0; u < DH / 8; ++u)
+                    d4[u * a.H_q] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+            }
+            if (store) a.lse_part[(prow * a.k + slot) * a.H_q + h] = lse_row;
             if (row == 0) TL(7, qt);
         }
     }
@@ -515,9 +604,9 @@ template <int DH, int G>
 cudaError_t launch_cfg(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
                        cudaStream_t s, int n_sm)
 {
-    using C = AttnCfg<DH>;
+    using C = AttnCfg<DH, G>;
     const int smem = C::SMEM + (int)sizeof(AttnShared);
-    static_assert(AttnCfg<DH>::SMEM + sizeof(AttnShared) <= 227 * 1024, "shared memory budget");
+    static_assert(C::SMEM + sizeof(AttnShared) <= 227 * 1024, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     sparse_attn_kernel<DH, G><<<n_sm, 512, smem, s>>>(a, qmap, kmap, vmap);
