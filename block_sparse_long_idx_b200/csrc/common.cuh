@@ -96,8 +96,8 @@ struct AttnArgs {
     const int32_t* blk_qtok = nullptr; // packed batch: query-row coordinate of each block's first token
                                        // (differs from blk_tok when keys and queries are packed apart)
     long long* timeline;        // optional: CTA 0 records clock64 per tile event (nullptr = off)
-    int timeline_tiles;         // capacity in tiles (16 event slots per tile)
-    uint16_t* o_part;           // [rows][k][H_q][d_h]
+    int timeline_tiles;         // capacity in tiles (48 event slots per tile)
+    uint16_t* o_part;           // [rows][k][d_h / 8][H_q][8] bf16 (normalised partial outputs)
     float* lse_part;            // [rows][k][H_q]
     int* err;
 };

@@ -17,7 +17,7 @@
 // Roles (512 threads, four warpgroups):
 //   WG0: warp 0 = K/V TMA producer, warp 1 = S issuer + TMEM owner, warp 2 = tile scheduler and Q
 //        gather (TMA boxes issued by the 32 lanes in parallel), warp 3 = PV issuer
-//   WG1, WG2: softmax of even / odd tiles
+//   WG1, WG2: softmax, one 64-column half of every tile each
 //   WG3: epilogue of every tile (O / rowsum -> partial slot)
 // Work items are claimed dynamically: the tile scheduler takes the next item of the launch's work
 // list from a global atomic counter (so CTAs that drew short items take more), one item ahead of
@@ -33,17 +33,21 @@
 // while its output columns are busy only from PV until the epilogue has read them, so TMEM (512
 // columns) holds three S/P regions R[t % 3] at columns 0, 128, 256 (S, then P in the first 64
 // columns) and one output region at columns 384-511: three tiles are in flight between S and PV.
-// Two threads issue the MMAs: the S issuer issues S(t) once PV(t-3) has consumed P(t-3) (region
-// R[t % 3] free) and Q(t) has landed; the PV issuer issues PV(t) once P(t) is written and the
-// epilogue has read O(t-1). Q has three shared-memory stages (stage t % 3, refilled for t+3 once
-// S(t) has completed). K and V of consecutive items rotate through three 128-row buffers in load
-// order K0 V0 K1 V1 ...: load n goes to buffer n % 3 once load n-3 is released (the K of an item
-// after its last S, its V after its last PV), so the next item's K and V stream in while the
-// current item's tiles run.
-// Barriers: s_full, p_full, pv_done per S/P region; o_full, o_free for the output region; ml_full[4]
-// hands each tile's lse and 1 / (rounded row sum) from the softmax to the epilogue through shared memory
-// (slot t % 4, rewritten by the softmax of t+4, which needs S(t+4), which needs PV(t+1), which needs
-// the epilogue of t to have read O(t), after it read the slot).
+// Both softmax warpgroups work on every tile (one 64-column half of the keys each, exchanging the
+// row maxima through shared memory), which halves a tile's softmax latency.
+// Two threads issue the MMAs. A thread stays busy about as long as the tensor pipe takes to run
+// what it issues, and every barrier wait or tcgen05.commit costs it tens of cycles, so each issuer
+// reads only the first record of an item (which carries the item's tile count) and per tile waits
+// on two barriers and commits one: the S issuer waits for Q(t) and for PV(t-3) (region R[t % 3]
+// free) and commits s_full, which also frees Q stage t % 3; the PV issuer waits for P(t) and for the
+// epilogue's read of O(t-1) and commits pv_done, which frees region R[t % 3] and hands O(t) to the
+// epilogue. Q has three shared-memory stages (stage t % 3, refilled for t+3 once S(t) completed).
+// K and V of consecutive items rotate through three 128-row buffers in load order K0 V0 K1 V1 ...:
+// load n goes to buffer n % 3 once load n-3 is released (the K of an item after its last S, its V
+// after its last PV), so the next item's K and V stream in while the current item's tiles run.
+// The softmax hands each tile's row max and row sums to the epilogue through shared memory (slot
+// t % 4, ml_full[t % 4]; rewritten by the softmax of t+4, which needs S(t+4), which needs PV(t+1),
+// which needs the epilogue of t to have read O(t), after it read the slot).
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -75,21 +79,22 @@ constexpr int kRegions = 3; // S/P regions in TMEM
 constexpr uint32_t kOCol = 384;
 
 struct TileRec {
-    int32_t r, b;  // GQA group, KV block
-    int32_t npos;  // positions in the tile (1 .. 128/G); -1 marks the end of the CTA's work
-    int32_t flags; // bit 0: first tile of its item, bit 1: last tile
-    int32_t tok0;  // query-row coordinate of block b's first token (b * 128 for one sequence)
+    int32_t r, b;   // GQA group, KV block
+    int32_t npos;   // positions in the tile (1 .. 128/G); -1 marks the end of the CTA's work
+    int32_t flags;  // bit 0: first tile of its item, bit 1: last tile
+    int32_t tok0;   // query-row coordinate of block b's first token (b * 128 for one sequence)
+    int32_t ntiles; // tiles of the item (the MMA issuers read only each item's first record)
 };
 
 struct AttnShared {
     uint64_t kv_full[3], kv_empty[3];
-    uint64_t q_full[3], q_empty[3];
+    uint64_t q_full[3];
     uint64_t s_full[kRegions], p_full[kRegions], pv_done[kRegions];
-    uint64_t o_full, o_free;
+    uint64_t o_free;
     uint64_t ml_full[4];
     uint64_t tile_full[kRing], tile_free[kRing];
     uint64_t kvrec_full[4], kvrec_free[4];
-    uint64_t done;
+    uint64_t done, done2;
     uint64_t xbar[2][4];    // [tile & 1][lane quarter]: both softmax warps of the quarter hold their max
     float xmax[2][2][128];  // [tile & 1][column half][row]: the halves' row maxima, exchanged
     float mrow[4][128];     // [tile slot][row]: row max of the raw scores
@@ -132,7 +137,7 @@ __global__ void __launch_bounds__(512, 1)
     const bool tl_on = a.timeline != nullptr && cta == 0;
 #define TL(slot, tile)                                                                                    \
     do {                                                                                                  \
-        if (tl_on && (tile) < a.timeline_tiles) a.timeline[(int64_t)(tile) * 32 + (slot)] = clock64();    \
+        if (tl_on && (tile) < a.timeline_tiles) a.timeline[(int64_t)(tile) * 48 + (slot)] = clock64();    \
     } while (0)
 
     if (threadIdx.x == 0) {
@@ -145,12 +150,8 @@ __global__ void __launch_bounds__(512, 1)
             mbar_init(&sh.p_full[i], 8);
             mbar_init(&sh.pv_done[i], 1);
         }
-        mbar_init(&sh.o_full, 1);
         mbar_init(&sh.o_free, 4);
-        for (int i = 0; i < NQ; ++i) {
-            mbar_init(&sh.q_full[i], 1);
-            mbar_init(&sh.q_empty[i], 1);
-        }
+        for (int i = 0; i < NQ; ++i) mbar_init(&sh.q_full[i], 1);
         for (int i = 0; i < 4; ++i) mbar_init(&sh.ml_full[i], 8);
         for (int i = 0; i < 8; ++i) mbar_init(&sh.xbar[i >> 2][i & 3], 2);
         for (int i = 0; i < kRing; ++i) {
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(512, 1)
             mbar_init(&sh.kvrec_free[i], 1);
         }
         mbar_init(&sh.done, 1);
+        mbar_init(&sh.done2, 1);
         sh.abort_flag = 0;
         fence_mbar_init();
     }
@@ -266,11 +268,13 @@ __global__ void __launch_bounds__(512, 1)
                         if (pl < npos) sh.rec_e[rs][pl] = e[u];
                     }
                     if (lane == 0)
-                        sh.rec[rs] = TileRec{item.r, item.b, npos, (t == 0 ? 1 : 0) | (t == ntiles - 1 ? 2 : 0), tok0};
+                        sh.rec[rs] = TileRec{item.r, item.b, npos, (t == 0 ? 1 : 0) | (t == ntiles - 1 ? 2 : 0), tok0,
+                                             ntiles};
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh.tile_full[rs]);
+                    // Q stage qs is free once S(qt-3), the last reader of the stage, has completed
                     if (lane == 0)
-                        w_ok = wait_or_abort(&sh.q_empty[qs], ((qt / NQ) & 1) ^ 1, abort_flag, a.err, 21, kWaitLimit);
+                        w_ok = wait_or_abort(&sh.s_full[qs], ((qt / NQ) & 1) ^ 1, abort_flag, a.err, 21, kWaitLimit);
                     w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
                     if (!w_ok) {
                         ok = false;
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(512, 1)
                 const int rs = qt % kRing;
                 if (qt < kRing ||
                     wait_or_abort(&sh.tile_free[rs], ((qt / kRing) & 1) ^ 1, abort_flag, a.err, 33, kWaitLimit)) {
-                    sh.rec[rs] = TileRec{0, 0, -1, 0, 0};
+                    sh.rec[rs] = TileRec{0, 0, -1, 0, 0, 0};
                     mbar_arrive(&sh.tile_full[rs]);
                 }
             }
@@ -316,128 +320,94 @@ __global__ void __launch_bounds__(512, 1)
                 for (int g = n_tiles - 1; g >= 0 && g >= n_tiles - NQ; --g)
                     drain_wait(&sh.q_full[g % NQ], (g / NQ) & 1, a.err, 41, kWaitLimit);
         } else if (warp == 1) {
-            // -------------------------------------------------------- MMA issuer (S and PV)
-            // One thread issues every MMA. A ready PV goes first: it gates the epilogue, the output
-            // region and the S/P region of the tile three ahead, while an S issued early only waits
-            // in the tensor pipe. S(ts) needs its record, Q(ts), the item's K and PV(ts-3) complete;
-            // PV(tp) needs S(tp) issued, P(tp), the item's V and the epilogue's read of O(tp-1).
+            // -------------------------------------------------------- S issuer: S(t) = Q K^T
+            // reads only each item's first record; per tile it waits for Q(t) and for PV(t-3) to have
+            // consumed P(t-3) (region R[t % 3] free), and commits one barrier (s_full, which also
+            // frees Q stage t % 3 for the scheduler)
             if (lane == 0) {
                 constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
-                constexpr uint32_t idPV = idesc_bf16_f32(128, DH, true);
                 const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV);
-                int ts = 0, tp = 0;     // next tile for S, for PV
-                int its = -1, itp = -1; // item counters of the two sides
-                int kb = 0, vb = 0;
-                bool s_rec = false, p_rec = false, s_end = false, p_end = false;
-                bool s_kv = false, p_kv = false; // the K (V) of the pending tile's item has landed
-                bool p_pf = false, p_of = false; // P(tp) written, O(tp-1) read
-                bool s_q = false, s_pv = false;  // Q(ts) landed, PV(ts-3) complete
-                TileRec rs_{}, rp_{};
-                uint64_t kdesc = 0, vdesc = 0;
-                long long t_last = clock64();
-                while (!(s_end && p_end)) {
-                    bool progress = false;
-                    // ---------------- PV(tp)
-                    if (!p_end && tp < ts) {
-                        if (!p_rec && mbar_poll(&sh.tile_full[tp % kRing], (tp / kRing) & 1)) {
-                            rp_ = sh.rec[tp % kRing];
-                            p_rec = true;
-                            if (rp_.flags & 1) {
-                                ++itp;
-                                vb = (2 * itp + 1) % NKV;
-                                p_kv = false;
-                            }
-                        }
-                        if (p_rec && !p_kv && mbar_poll(&sh.kv_full[vb], ((2 * itp + 1) / NKV) & 1)) {
-                            p_kv = true;
-                            vdesc = smem_desc(aKV + vb * C::TILE, C::CHUNK, 1024, 128);
-                        }
-                        const int reg = tp % kRegions;
-                        if (p_rec && !p_pf && mbar_poll(&sh.p_full[reg], (tp / kRegions) & 1)) {
-                            p_pf = true;
-                            TL(10, tp);
-                        }
-                        if (p_rec && !p_of && mbar_poll(&sh.o_free, (tp & 1) ^ 1)) {
-                            p_of = true;
-                            TL(11, tp);
-                        }
-                        if (p_rec && p_kv && p_pf && p_of) {
-                            TL(12, tp);
-                            tc_fence_after();
-                            const uint32_t acol = tmem + a_col(tp);
-#pragma unroll
-                            for (int ks = 0; ks < 8; ++ks) // 16 keys = 2048 bytes of V per step
-                                mma_ts(tmem + kOCol, acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
-                            tc_commit(&sh.pv_done[reg]);
-                            tc_commit(&sh.o_full);
-                            if (rp_.flags & 2) tc_commit(&sh.kv_empty[vb]); // the item's V is no longer read
-                            TL(3, tp);
-                            ++tp;
-                            p_rec = p_pf = p_of = false;
-                            progress = true;
-                        }
-                    } else if (!p_end && s_end && tp == ts) {
-                        p_end = true; // every issued S has its PV
-                    }
-                    // ---------------- S(ts)
-                    if (!s_end) {
-                        if (!s_rec && mbar_poll(&sh.tile_full[ts % kRing], (ts / kRing) & 1)) {
-                            rs_ = sh.rec[ts % kRing];
-                            s_rec = true;
-                            if (rs_.npos < 0) {
-                                s_end = true;
-                            } else if (rs_.flags & 1) {
-                                ++its;
-                                kb = (2 * its) % NKV;
-                                s_kv = false;
-                            }
-                        }
-                        if (s_rec && !s_end && !s_kv && mbar_poll(&sh.kv_full[kb], ((2 * its) / NKV) & 1)) {
-                            s_kv = true;
-                            kdesc = desc_kmajor(aKV + kb * C::TILE, 128);
-                            TL(8, ts);
-                        }
-                        const int reg = ts % kRegions, qs = ts % NQ;
-                        // region R[ts % 3] is free once PV(ts-3) has consumed P(ts-3)
-                        if (s_rec && !s_end && !s_q && mbar_poll(&sh.q_full[qs], (ts / NQ) & 1)) s_q = true;
-                        if (s_rec && !s_end && !s_pv && mbar_poll(&sh.pv_done[reg], ((ts / kRegions) & 1) ^ 1))
-                            s_pv = true;
-                        if (s_rec && !s_end && s_kv && s_q && s_pv) {
-                            TL(9, ts);
-                            tc_fence_after();
-                            const uint64_t qdesc = smem_desc(aQ + qs * C::TILE, 16, C::QSBO, 128);
-                            const uint32_t sd = tmem + a_col(ts);
-#pragma unroll
-                            for (int ks = 0; ks < DH / 16; ++ks) {
-                                const uint64_t qoff = (uint64_t)((((ks >> 2) * C::QCHUNK) + (ks & 3) * 32) >> 4);
-                                const uint64_t koff = (uint64_t)((((ks >> 2) * C::CHUNK) + (ks & 3) * 32) >> 4);
-                                mma_ss(sd, qdesc + qoff, kdesc + koff, idS, ks > 0);
-                            }
-                            tc_commit(&sh.s_full[reg]);
-                            tc_commit(&sh.q_empty[qs]);
-                            if (rs_.flags & 2) tc_commit(&sh.kv_empty[kb]); // the item's K is no longer read
-                            TL(2, ts);
-                            ++ts;
-                            s_rec = s_q = s_pv = false;
-                            progress = true;
-                        }
-                    }
-                    if (progress) {
-                        t_last = clock64();
-                    } else {
-                        // back off briefly: a spinning thread takes issue slots from the softmax and
-                        // epilogue warps of its SM sub-partition, which produce the next events
-                        __nanosleep(32);
-                        if (*abort_flag) break;
-                        if (clock64() - t_last > kWaitLimit) {
-                            report_error(a.err, MSA_ERR_TIMEOUT, 25);
-                            *abort_flag = 1;
+                int qt = 0;
+                bool ok = true;
+                for (int it = 0; ok; ++it) {
+                    const int rs = qt % kRing;
+                    if (!wait_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 34, kWaitLimit)) break;
+                    const TileRec rec = sh.rec[rs];
+                    if (rec.npos < 0) break;
+                    const int kb = (2 * it) % NKV; // K of item it = load 2*it
+                    if (!wait_or_abort(&sh.kv_full[kb], ((2 * it) / NKV) & 1, abort_flag, a.err, 23, kWaitLimit)) break;
+                    const uint64_t kdesc = desc_kmajor(aKV + kb * C::TILE, 128);
+                    TL(8, qt);
+                    for (int t = 0; t < rec.ntiles; ++t, ++qt) {
+                        const int reg = qt % kRegions;
+                        if (!wait_or_abort(&sh.q_full[reg], (qt / NQ) & 1, abort_flag, a.err, 24, kWaitLimit)) {
+                            ok = false;
                             break;
                         }
+                        TL(38, qt);
+                        if (!wait_or_abort(&sh.pv_done[reg], ((qt / kRegions) & 1) ^ 1, abort_flag, a.err, 25,
+                                           kWaitLimit)) {
+                            ok = false;
+                            break;
+                        }
+                        TL(9, qt);
+                        tc_fence_after();
+                        const uint64_t qdesc = smem_desc(aQ + reg * C::TILE, 16, C::QSBO, 128);
+                        const uint32_t sd = tmem + a_col(qt);
+#pragma unroll
+                        for (int ks = 0; ks < DH / 16; ++ks) {
+                            const uint64_t qoff = (uint64_t)((((ks >> 2) * C::QCHUNK) + (ks & 3) * 32) >> 4);
+                            const uint64_t koff = (uint64_t)((((ks >> 2) * C::CHUNK) + (ks & 3) * 32) >> 4);
+                            mma_ss(sd, qdesc + qoff, kdesc + koff, idS, ks > 0);
+                        }
+                        TL(32, qt);
+                        tc_commit(&sh.s_full[reg]);
+                        if (t == rec.ntiles - 1) tc_commit(&sh.kv_empty[kb]); // the item's K is no longer read
+                        TL(2, qt);
                     }
                 }
                 tc_commit(&sh.done);
                 drain_wait(&sh.done, 0, a.err, 42, kWaitLimit);
+            }
+        } else if (warp == 3) {
+            // -------------------------------------------------------- PV issuer: O(t) = P(t) V
+            // reads only each item's first record; per tile it waits for P(t) and for the epilogue's
+            // read of O(t-1), and commits one barrier (pv_done: region R[t % 3] free, O(t) ready)
+            if (lane == 0) {
+                constexpr uint32_t idPV = idesc_bf16_f32(128, DH, true);
+                const uint32_t aKV = smem_u32(sKV);
+                int qt = 0;
+                bool ok = true;
+                for (int it = 0; ok; ++it) {
+                    const int rs = qt % kRing;
+                    if (!wait_or_abort(&sh.tile_full[rs], (qt / kRing) & 1, abort_flag, a.err, 35, kWaitLimit)) break;
+                    const TileRec rec = sh.rec[rs];
+                    if (rec.npos < 0) break;
+                    const int vb = (2 * it + 1) % NKV; // V of item it = load 2*it + 1
+                    if (!wait_or_abort(&sh.kv_full[vb], ((2 * it + 1) / NKV) & 1, abort_flag, a.err, 30, kWaitLimit))
+                        break;
+                    const uint64_t vdesc = smem_desc(aKV + vb * C::TILE, C::CHUNK, 1024, 128);
+                    for (int t = 0; t < rec.ntiles; ++t, ++qt) {
+                        const int reg = qt % kRegions;
+                        if (!wait_or_abort(&sh.p_full[reg], (qt / kRegions) & 1, abort_flag, a.err, 22, kWaitLimit) ||
+                            !wait_or_abort(&sh.o_free, (qt & 1) ^ 1, abort_flag, a.err, 28, kWaitLimit)) {
+                            ok = false;
+                            break;
+                        }
+                        TL(12, qt);
+                        tc_fence_after();
+                        const uint32_t acol = tmem + a_col(qt);
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks) // 16 keys = 2048 bytes of V per step
+                            mma_ts(tmem + kOCol, acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
+                        TL(36, qt);
+                        tc_commit(&sh.pv_done[reg]);
+                        if (t == rec.ntiles - 1) tc_commit(&sh.kv_empty[vb]); // the item's V is no longer read
+                        TL(3, qt);
+                    }
+                }
+                tc_commit(&sh.done2);
+                drain_wait(&sh.done2, 0, a.err, 43, kWaitLimit);
             }
         }
     } else if (wg <= 2) {
@@ -489,6 +459,7 @@ __global__ void __launch_bounds__(512, 1)
             if (lane == 0) mbar_arrive(&sh.xbar[qt & 1][quarter]);
             if (!wait_or_abort(&sh.xbar[qt & 1][quarter], (qt >> 1) & 1, abort_flag, a.err, 44, kWaitLimit)) break;
             tc_fence_after();
+            if (row == 0 && beta == 0) TL(33, qt);
             const float m = fmaxf(sh.xmax[qt & 1][0][row], sh.xmax[qt & 1][1][row]);
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t nmx2 = f2_pack(-m * sl2, -m * sl2);
@@ -512,7 +483,9 @@ __global__ void __launch_bounds__(512, 1)
             // that the PV product uses normalises O, so each partial is an exact weighted average
             sh.lsum[qt & 3][beta][row] = make_float2(f2_lo(l2) + f2_hi(l2), f2_lo(lr2) + f2_hi(lr2));
             if (beta == 0) sh.mrow[qt & 3][row] = m;
+            if (row == 0 && beta == 0) TL(34, qt);
             tmem_st_wait();
+            if (row == 0 && beta == 0) TL(35, qt);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -540,7 +513,7 @@ __global__ void __launch_bounds__(512, 1)
             const int32_t e = valid ? sh.rec_e[rs][pl] : 0;
             const int p = e / a.k;
             const int slot = e - p * a.k;
-            if (!wait_or_abort(&sh.o_full, qt & 1, abort_flag, a.err, 27, kWaitLimit) ||
+            if (!wait_or_abort(&sh.pv_done[qt % kRegions], (qt / kRegions) & 1, abort_flag, a.err, 27, kWaitLimit) ||
                 !wait_or_abort(&sh.ml_full[qt & 3], (qt >> 2) & 1, abort_flag, a.err, 29, kWaitLimit))
                 break;
             if (row == 0) TL(6, qt);
