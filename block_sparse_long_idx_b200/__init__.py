@@ -8,7 +8,8 @@ _API_NAMES = {
     "lib", "LIB_PATH", "MsaError", "KV2Q", "msa_kv2q_layout", "status_string", "msa_get_device_error",
     "msa_index_topk", "msa_kv2q_layout_get", "msa_build_kv2q", "msa_sparse_prefill_workspace_size",
     "msa_sparse_prefill", "msa_sparse_decode", "SIGNATURES", "KernelTrace", "msa_launch_count", "KERNEL_NAMES",
-    "msa_selftest_wait_timeout", "msa_sparse_prefill_varlen", "msa_sparse_backward",
+    "msa_selftest_wait_timeout", "msa_sparse_prefill_varlen", "msa_sparse_backward", "msa_quantize_e4m3",
+    "msa_sparse_prefill_fp8", "E4M3Rows",
 }
 
 

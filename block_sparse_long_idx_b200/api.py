@@ -61,6 +61,9 @@ SIGNATURES = [
     ("msa_sparse_backward_workspace_size", _sz, [_i64, _int, _int, _int, _int, _int, _int, _int]),
     ("msa_sparse_backward", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _int, _int, _vp, _LP, _vp,
                                    _vp, _vp, _vp, _vp, _vp, _int, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
+    ("msa_quantize_e4m3", _int, [_vp, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp]),
+    ("msa_sparse_prefill_fp8", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _int, _int,
+                                      _vp, _LP, _vp, _vp, _vp, _vp, _sz, _vp]),
     ("msa_selftest_workspace_size", _sz, []),
     ("msa_selftest_wait_timeout", _int, [_vp, _sz, _i64, _vp]),
     ("msa_trace_set", None, [_vp]),
@@ -363,3 +366,49 @@ def msa_sparse_decode(q, q_idx, k_cache, v_cache, k_idx_cache, lens, B_k: int = 
         lens.data_ptr(), B, L_max, H_q, H_kv, d_h, d_idx, B_k, k, out.data_ptr(), _ptr(lse),
         block_idx_out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)))
     return out, lse, block_idx_out
+
+
+class E4M3Rows:
+    """Per-row E4M3 quantisation of a [N, H, d] tensor: codes [N, H, d] uint8, scales and rscales
+    [H, S] float32 (S = N rounded up to whole 128-token blocks), blkmax [H, S / 128] float32."""
+
+    def __init__(self, codes, scales, rscales, blkmax):
+        self.codes, self.scales, self.rscales, self.blkmax = codes, scales, rscales, blkmax
+
+
+def msa_quantize_e4m3(x, with_rscales: bool = True, with_blkmax: bool = True, stream=None) -> E4M3Rows:
+    """E4M3 codes and per-row scales (amax / 448) of x [N, H, d] bf16."""
+    _bf16(x, "x")
+    N, H, d = x.shape
+    S = (N + 127) // 128 * 128
+    codes = torch.empty((N, H, d), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((H, S), dtype=torch.float32, device=x.device)
+    rscales = torch.empty((H, S), dtype=torch.float32, device=x.device) if with_rscales else None
+    blkmax = torch.empty((H, S // 128), dtype=torch.float32, device=x.device) if with_blkmax else None
+    _check("msa_quantize_e4m3", lib.msa_quantize_e4m3(x.data_ptr(), N, H, d, codes.data_ptr(), scales.data_ptr(),
+                                                       _ptr(rscales), _ptr(blkmax), _stream(stream)))
+    return E4M3Rows(codes, scales, rscales, blkmax)
+
+
+def msa_sparse_prefill_fp8(q8: E4M3Rows, k8: E4M3Rows, v8: E4M3Rows, block_idx, kv2q: KV2Q | None = None,
+                           B_k: int = 128, out=None, lse=None, want_lse: bool = True, workspace=None,
+                           max_rows_per_pass: int = 0, stream=None):
+    """FP8 main branch on E4M3 codes and scales from msa_quantize_e4m3. Returns (out bf16, lse)."""
+    N, H_q, d_h = q8.codes.shape
+    H_kv = k8.codes.shape[1]
+    kk = block_idx.shape[2]
+    if out is None:
+        out = torch.empty((N, H_q, d_h), dtype=torch.bfloat16, device=q8.codes.device)
+    if lse is None and want_lse:
+        lse = torch.empty((N, H_q), dtype=torch.float32, device=q8.codes.device)
+    if workspace is None:
+        workspace = torch.empty(msa_sparse_prefill_workspace_size(N, H_q, H_kv, d_h, B_k, kk, max_rows_per_pass,
+                                                                  kv2q is None), dtype=torch.uint8,
+                                device=q8.codes.device)
+    lp = ctypes.byref(kv2q.layout) if kv2q is not None else None
+    _check("msa_sparse_prefill_fp8", lib.msa_sparse_prefill_fp8(
+        q8.codes.data_ptr(), q8.scales.data_ptr(), k8.codes.data_ptr(), k8.scales.data_ptr(), v8.codes.data_ptr(),
+        v8.scales.data_ptr(), v8.rscales.data_ptr(), v8.blkmax.data_ptr(), N, H_q, H_kv, d_h, B_k, kk,
+        block_idx.data_ptr(), lp, _ptr(kv2q.buf) if kv2q is not None else None, out.data_ptr(), _ptr(lse),
+        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out, lse

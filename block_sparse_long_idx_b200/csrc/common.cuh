@@ -100,12 +100,37 @@ struct AttnArgs {
     uint16_t* o_part;           // [rows][k][d_h / 8][H_q][8] bf16 (normalised partial outputs)
     float* lse_part;            // [rows][k][H_q]
     int* err;
+    // FP8 main branch (the q, k, v maps then hold E4M3 codes): head-major row scales [H][sstride]
+    const float* qs = nullptr;      // q scales
+    const float* ks = nullptr;      // k scales
+    const float* vs = nullptr;      // v scales
+    const float* rvs = nullptr;     // reciprocals of the v scales
+    const float* vblkmax = nullptr; // [H_kv][nb]: largest v scale of each 128-token block
+    int64_t sstride = 0;            // N rounded up to whole 128-token blocks
+    int nb = 0;
 };
+
+// Per-row E4M3 quantisation: x [N][H][d] bf16 -> codes [N][H][d], scales [H][N_pad] (amax / 448, 1 for
+// an all-zero or padding row), rscales = 1 / scales (nullable), blkmax [H][nb] = largest scale of each
+// 128-token block (nullable; zeroed by the caller).
+struct QuantArgs {
+    const uint16_t* x;
+    int64_t N, N_pad;
+    int H, d, nb;
+    uint8_t* codes;
+    float* scales;
+    float* rscales;
+    float* blkmax;
+};
+cudaError_t launch_quantize_e4m3(const QuantArgs& a, cudaStream_t s);
 // One thread waits on a barrier phase that never completes; the wait expires after limit_cycles.
 cudaError_t launch_selftest_wait(int* err, long long limit_cycles, cudaStream_t s);
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                                const CUtensorMap& vmap, cudaStream_t s);
+// The same on E4M3 codes (d_h = 128): the maps describe 8-bit tensors, a.qs .. a.vblkmax are set.
+cudaError_t launch_sparse_attn_fp8(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                                   const CUtensorMap& vmap, cudaStream_t s);
 
 struct CombineArgs {
     int64_t row0, n_rows; // rows [row0, row0+n_rows) of the sequence

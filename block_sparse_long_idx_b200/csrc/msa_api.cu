@@ -34,18 +34,18 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 3-D bf16 tensor [n2][n1][n0] (row-major), box {b0, b1, b2}.
+// 3-D tensor [n2][n1][n0] (row-major) of bf16 (eb = 2) or 8-bit codes (eb = 1), box {b0, b1, b2}.
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t b0, uint32_t b1,
-                 uint32_t b2, CUtensorMapSwizzle sw)
+                 uint32_t b2, CUtensorMapSwizzle sw, int eb = 2)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {n0, n1, n2};
-    const cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+    const cuuint64_t strides[2] = {n0 * eb, n0 * n1 * eb};
     const cuuint32_t box[3] = {b0, b1, b2};
     const cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(m, eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base),
+              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -54,19 +54,21 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uin
 // of 8, position), so the box lands in shared memory as [head group][chunk][8 heads][128 B] and the
 // tile's 8-row groups are a uniform 1024 * d_h / 64 bytes apart. G < 8: one 3-D box of G heads x 64
 // columns per 64-column chunk.
-bool make_qmap(CUtensorMap* m, const void* q, int d_h, int H_q, int64_t N, int G)
+bool make_qmap(CUtensorMap* m, const void* q, int d_h, int H_q, int64_t N, int G, int eb = 2)
 {
-    if (G < 8) return make_map_3d(m, q, d_h, H_q, N, 64, G, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    const uint32_t ce = 128 / eb; // elements per 128-byte chunk
+    if (G < 8) return make_map_3d(m, q, d_h, H_q, N, ce, G, 1, CU_TENSOR_MAP_SWIZZLE_128B, eb);
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t nkc = (cuuint64_t)d_h / 64;
-    const cuuint64_t dims[5] = {64, 8, nkc, (cuuint64_t)H_q / 8, (cuuint64_t)N};
-    const cuuint64_t strides[4] = {(cuuint64_t)d_h * 2, 128, (cuuint64_t)8 * d_h * 2, (cuuint64_t)H_q * d_h * 2};
-    const cuuint32_t box[5] = {64, 8, (cuuint32_t)nkc, (cuuint32_t)(G / 8), 1};
+    const cuuint64_t nkc = (cuuint64_t)d_h / ce;
+    const cuuint64_t row = (cuuint64_t)d_h * eb;
+    const cuuint64_t dims[5] = {ce, 8, nkc, (cuuint64_t)H_q / 8, (cuuint64_t)N};
+    const cuuint64_t strides[4] = {row, 128, 8 * row, (cuuint64_t)H_q * row};
+    const cuuint32_t box[5] = {ce, 8, (cuuint32_t)nkc, (cuuint32_t)(G / 8), 1};
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(q), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(m, eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(q),
+              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -361,7 +363,8 @@ static msa_status run_passes(const uint8_t* kvb, const msa_kv2q_layout* L, int64
                              const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
                              int64_t wins_per_pass, int64_t rows_pass, uint16_t* o_part, float* lse_part,
                              msa_bf16* out, float* lse, void* workspace, cudaStream_t s, const int32_t* blk_tok,
-                             const int32_t* row_start, const int32_t* blk_qtok = nullptr)
+                             const int32_t* row_start, const int32_t* blk_qtok = nullptr,
+                             const AttnArgs* f8 = nullptr)
 {
     for (int64_t w0 = 0; w0 < L->n_windows; w0 += wins_per_pass) {
         const int64_t w1 = w0 + wins_per_pass < L->n_windows ? w0 + wins_per_pass : L->n_windows;
@@ -386,10 +389,20 @@ static msa_status run_passes(const uint8_t* kvb, const msa_kv2q_layout* L, int64
         a.o_part = o_part;
         a.lse_part = lse_part;
         a.err = (int*)workspace;
+        if (f8) {
+            a.qs = f8->qs;
+            a.ks = f8->ks;
+            a.vs = f8->vs;
+            a.rvs = f8->rvs;
+            a.vblkmax = f8->vblkmax;
+            a.sstride = f8->sstride;
+            a.nb = f8->nb;
+        }
         if (msa_status st1 = cuda_status(cudaMemsetAsync(a.item_counter, 0, sizeof(int), s), "clearing the work counter"))
             return st1;
         trace_begin(s);
-        const cudaError_t ea = launch_sparse_attn(a, qmap, kmap, vmap, s);
+        const cudaError_t ea = f8 ? launch_sparse_attn_fp8(a, qmap, kmap, vmap, s)
+                                  : launch_sparse_attn(a, qmap, kmap, vmap, s);
         trace_end(s, MSA_KERNEL_ATTN);
         if (ea != cudaSuccess) return cuda_status(ea, "attention launch");
         CombineArgs c;
@@ -488,6 +501,105 @@ msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* kk, const msa_b
     }
     return run_passes((const uint8_t*)kv, L, N, H_q, H_kv, d_h, k, qmap, kmap, vmap, wins_per_pass, rows_pass, o_part,
                       lse_part, out, lse, workspace, s, nullptr, nullptr);
+}
+
+// ------------------------------------------------------------------------------------ FP8 main branch
+msa_status msa_quantize_e4m3(const msa_bf16* x, int64_t N, int H, int d, uint8_t* codes, float* scales,
+                             float* rscales, float* blkmax, msa_stream_t stream)
+{
+    if (!x || !codes || !scales || N < 1 || H < 1 || d < 1) return MSA_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || (rscales && !aligned(rscales, 16)) ||
+        (blkmax && !aligned(blkmax, 4)))
+        return MSA_ERR_INVALID_ARG;
+    if (!(d == 64 || d == 128) || N > kMaxN) return MSA_ERR_UNSUPPORTED;
+    if (injected("msa_quantize_e4m3")) return MSA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    QuantArgs a;
+    a.x = x;
+    a.N = N;
+    a.nb = (int)((N + kBk - 1) / kBk);
+    a.N_pad = (int64_t)a.nb * kBk;
+    a.H = H;
+    a.d = d;
+    a.codes = codes;
+    a.scales = scales;
+    a.rscales = rscales;
+    a.blkmax = blkmax;
+    if (blkmax)
+        if (msa_status st = cuda_status(cudaMemsetAsync(blkmax, 0, (size_t)H * a.nb * 4, s), "clearing blkmax"))
+            return st;
+    return cuda_status(launch_quantize_e4m3(a, s), "quantize launch");
+}
+
+msa_status msa_sparse_prefill_fp8(const uint8_t* q8, const float* qs, const uint8_t* k8, const float* ks,
+                                  const uint8_t* v8, const float* vs, const float* rvs, const float* vblkmax, int64_t N,
+                                  int H_q, int H_kv, int d_h, int B_k, int k, const int32_t* block_idx,
+                                  const msa_kv2q_layout* layout, const void* kv2q, msa_bf16* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, msa_stream_t stream)
+{
+    if (!q8 || !qs || !k8 || !ks || !v8 || !vs || !rvs || !vblkmax || !block_idx || !out || !workspace || N < 1 ||
+        H_q < 1 || H_kv < 1 || d_h < 1 || k < 1)
+        return MSA_ERR_INVALID_ARG;
+    if ((layout == nullptr) != (kv2q == nullptr)) return MSA_ERR_INVALID_ARG;
+    if (H_q % H_kv != 0) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(qs, 16) || !aligned(ks, 16) ||
+        !aligned(vs, 16) || !aligned(rvs, 16) || !aligned(vblkmax, 4) || !aligned(out, 16) || !aligned(workspace, 256) ||
+        (lse && !aligned(lse, 4)))
+        return MSA_ERR_INVALID_ARG;
+    const int G = H_q / H_kv;
+    if (B_k != kBk || k > kMaxK || d_h != 128 || !pow2(G) || G > 16 || N > kMaxN) return MSA_ERR_UNSUPPORTED;
+    if (layout && (!layout_ok(layout) || layout->N != N || layout->H_kv != H_kv || layout->k != k))
+        return MSA_ERR_INVALID_ARG;
+    if (injected("msa_sparse_prefill_fp8")) return MSA_ERR_CUDA;
+
+    msa_kv2q_layout Lint;
+    const msa_kv2q_layout* L = layout;
+    uint8_t* ws = (uint8_t*)workspace;
+    size_t used = kErrBytes;
+    const void* kv = kv2q;
+    cudaStream_t s = (cudaStream_t)stream;
+    void* kvbuf = nullptr;
+    void* kvtmp = nullptr;
+    if (!L) {
+        msa_kv2q_layout_get(N, H_kv, B_k, k, 0, 0, &Lint);
+        L = &Lint;
+        const size_t need = align_up(L->total_bytes, 256) + align_up(kv2q_internal_tmp(*L), 256);
+        if (workspace_bytes < used + need) return MSA_ERR_WORKSPACE;
+        kvbuf = ws + used;
+        kvtmp = ws + used + align_up(L->total_bytes, 256);
+        used += need;
+        kv = kvbuf;
+    }
+    const size_t per_row = partial_row_bytes(H_q, d_h, k);
+    if (workspace_bytes <= used + 512) return MSA_ERR_WORKSPACE;
+    int64_t wins_per_pass = (int64_t)((workspace_bytes - used - 512) / per_row) / L->window;
+    if (wins_per_pass < 1) return MSA_ERR_WORKSPACE;
+    if (wins_per_pass > L->n_windows) wins_per_pass = L->n_windows;
+    const int64_t rows_pass = wins_per_pass * L->window;
+    uint16_t* o_part = (uint16_t*)(ws + used);
+    float* lse_part = (float*)(ws + used + align_up((size_t)rows_pass * k * H_q * d_h * 2, 256));
+
+    CUtensorMap qmap, kmap, vmap;
+    if (!make_qmap(&qmap, q8, d_h, H_q, N, G, 1) ||
+        !make_map_3d(&kmap, k8, d_h, H_kv, N, 128, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B, 1) ||
+        !make_map_3d(&vmap, v8, d_h, H_kv, N, 128, 1, kBk, CU_TENSOR_MAP_SWIZZLE_128B, 1))
+        return MSA_ERR_INVALID_ARG;
+    AttnArgs f8;
+    f8.qs = qs;
+    f8.ks = ks;
+    f8.vs = vs;
+    f8.rvs = rvs;
+    f8.vblkmax = vblkmax;
+    f8.nb = (int)((N + kBk - 1) / kBk);
+    f8.sstride = (int64_t)f8.nb * kBk;
+
+    if (msa_status st0 = cuda_status(cudaMemsetAsync(workspace, 0, kErrBytes, s), "clearing the error word")) return st0;
+    if (kvbuf) {
+        msa_status st = build_kv2q_impl(block_idx, L, kvbuf, (int*)workspace, kvtmp, s);
+        if (st != MSA_OK) return st;
+    }
+    return run_passes((const uint8_t*)kv, L, N, H_q, H_kv, d_h, k, qmap, kmap, vmap, wins_per_pass, rows_pass, o_part,
+                      lse_part, out, lse, workspace, s, nullptr, nullptr, nullptr, &f8);
 }
 
 // ------------------------------------------------------------------------------------ backward

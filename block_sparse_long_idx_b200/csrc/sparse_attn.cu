@@ -57,9 +57,12 @@ namespace msa {
 
 namespace {
 
-template <int DH, int G>
+template <int DH, int G, bool F8>
 struct AttnCfg {
-    static constexpr int NKC = DH / 64;          // 64-column (128-byte) chunks
+    static constexpr int EB = F8 ? 1 : 2;        // bytes per operand element (E4M3 or bf16)
+    static constexpr int NKC = DH * EB / 128;    // 128-byte chunks of an operand row
+    static constexpr int CE = 128 / EB;          // elements per chunk
+    static constexpr int KSTEPS = DH * EB / 32;  // S MMAs per tile (32 bytes of K each)
     static constexpr int CHUNK = 128 * 128;      // bytes per chunk of a 128-row tile
     static constexpr int TILE = NKC * CHUNK;     // Q, K or V tile bytes
     static constexpr int NQ = 3;                 // Q stages
@@ -71,7 +74,7 @@ struct AttnCfg {
     // (position, chunk).
     static constexpr bool QPOS = G >= 8;
     static constexpr int QSBO = QPOS ? NKC * 1024 : 1024; // bytes between 8-row groups
-    static constexpr int QCHUNK = QPOS ? 1024 : CHUNK;    // bytes between 64-column chunks
+    static constexpr int QCHUNK = QPOS ? 1024 : CHUNK;    // bytes between 128-byte chunks
 };
 
 constexpr int kRing = 8;    // tile records in flight between the scheduler and the epilogue
@@ -84,6 +87,7 @@ struct TileRec {
     int32_t flags;  // bit 0: first tile of its item, bit 1: last tile
     int32_t tok0;   // query-row coordinate of block b's first token (b * 128 for one sequence)
     int32_t ntiles; // tiles of the item (the MMA issuers read only each item's first record)
+    int32_t item;   // the CTA's item counter (K of item i is load 2i, V load 2i+1, buffer = load % 3)
 };
 
 struct AttnShared {
@@ -102,6 +106,11 @@ struct AttnShared {
     TileRec rec[kRing];
     msa_work_item kvrec[4]; // items handed to the K/V producer (len = 0: no more work)
     int32_t rec_e[kRing][128]; // entry (i*k + slot) of each position of the tile
+    // FP8 only: per K/V buffer holding a V load, the item's k scales, v scales and their reciprocals
+    // (128 tokens each, loaded with V: the slot lives until the item's last PV) and 448 / (largest
+    // v scale of the block)
+    alignas(16) float fscl[3][3][128];
+    float fcb[3];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -113,12 +122,12 @@ static_assert(REG_PRODUCER + 2 * REG_SOFTMAX + REG_EPILOGUE <= 4 * REG_LAUNCH, "
 
 __device__ __forceinline__ uint32_t a_col(int t) { return (uint32_t)(t % kRegions) * 128; }
 
-template <int DH, int G>
+template <int DH, int G, bool F8>
 __global__ void __launch_bounds__(512, 1)
     sparse_attn_kernel(AttnArgs a, const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap)
 {
-    using C = AttnCfg<DH, G>;
+    using C = AttnCfg<DH, G, F8>;
     constexpr int PPT = 128 / G;
     constexpr int NQ = C::NQ, NKV = C::NKV;
     extern __shared__ uint8_t smem_raw[];
@@ -198,10 +207,24 @@ __global__ void __launch_bounds__(512, 1)
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&sh.kv_full[buf], C::TILE);
+                        if constexpr (F8) {
+                            if (kv) { // with V: the item's k, v, 1/v scales (512 B each) and 448 / block max
+                                const float vmax = a.vblkmax[(int64_t)item.r * a.nb + item.b];
+                                sh.fcb[buf] = vmax > 0.f ? 448.f / vmax : 1.f;
+                                mbar_arrive_expect_tx(&sh.kv_full[buf], C::TILE + 3 * 512);
+                                const int64_t so = (int64_t)item.r * a.sstride + tok0;
+                                bulk_load(sh.fscl[buf][0], a.ks + so, 512, &sh.kv_full[buf]);
+                                bulk_load(sh.fscl[buf][1], a.vs + so, 512, &sh.kv_full[buf]);
+                                bulk_load(sh.fscl[buf][2], a.rvs + so, 512, &sh.kv_full[buf]);
+                            } else {
+                                mbar_arrive_expect_tx(&sh.kv_full[buf], C::TILE);
+                            }
+                        } else {
+                            mbar_arrive_expect_tx(&sh.kv_full[buf], C::TILE);
+                        }
                         for (int c = 0; c < C::NKC; ++c)
                             tma_load_3d(sKV + buf * C::TILE + c * C::CHUNK, kv ? &vmap : &kmap, &sh.kv_full[buf],
-                                        c * 64, item.r, tok0);
+                                        c * C::CE, item.r, tok0);
                     }
                 }
                 for (int g = n - 1; g >= 0 && g >= n - NKV; --g)
@@ -269,7 +292,7 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     if (lane == 0)
                         sh.rec[rs] = TileRec{item.r, item.b, npos, (t == 0 ? 1 : 0) | (t == ntiles - 1 ? 2 : 0), tok0,
-                                             ntiles};
+                                             ntiles, it};
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh.tile_full[rs]);
                     // Q stage qs is free once S(qt-3), the last reader of the stage, has completed
@@ -282,7 +305,7 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     if (lane == 0) {
                         TL(0, qt);
-                        mbar_arrive_expect_tx(&sh.q_full[qs], npos * G * DH * 2);
+                        mbar_arrive_expect_tx(&sh.q_full[qs], npos * G * DH * C::EB);
                     }
                     __syncwarp();
 #pragma unroll
@@ -291,12 +314,12 @@ __global__ void __launch_bounds__(512, 1)
                         if (pl < npos) {
                             uint8_t* dst = sQ + qs * C::TILE;
                             if constexpr (C::QPOS) {
-                                tma_load_5d(dst + pl * (G * DH * 2), &qmap, &sh.q_full[qs], 0, 0, 0, item.r * (G / 8),
-                                            e[u] / a.k);
+                                tma_load_5d(dst + pl * (G * DH * C::EB), &qmap, &sh.q_full[qs], 0, 0, 0,
+                                            item.r * (G / 8), e[u] / a.k);
                             } else {
 #pragma unroll
                                 for (int c = 0; c < C::NKC; ++c)
-                                    tma_load_3d(dst + c * C::CHUNK + pl * G * 128, &qmap, &sh.q_full[qs], c * 64,
+                                    tma_load_3d(dst + c * C::CHUNK + pl * G * 128, &qmap, &sh.q_full[qs], c * C::CE,
                                                 item.r * G, e[u] / a.k);
                             }
                         }
@@ -312,7 +335,7 @@ __global__ void __launch_bounds__(512, 1)
                 const int rs = qt % kRing;
                 if (qt < kRing ||
                     wait_or_abort(&sh.tile_free[rs], ((qt / kRing) & 1) ^ 1, abort_flag, a.err, 33, kWaitLimit)) {
-                    sh.rec[rs] = TileRec{0, 0, -1, 0, 0, 0};
+                    sh.rec[rs] = TileRec{0, 0, -1, 0, 0, 0, 0};
                     mbar_arrive(&sh.tile_full[rs]);
                 }
             }
@@ -325,7 +348,7 @@ __global__ void __launch_bounds__(512, 1)
             // consumed P(t-3) (region R[t % 3] free), and commits one barrier (s_full, which also
             // frees Q stage t % 3 for the scheduler)
             if (lane == 0) {
-                constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
+                constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
                 const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV);
                 int qt = 0;
                 bool ok = true;
@@ -355,10 +378,13 @@ __global__ void __launch_bounds__(512, 1)
                         const uint64_t qdesc = smem_desc(aQ + reg * C::TILE, 16, C::QSBO, 128);
                         const uint32_t sd = tmem + a_col(qt);
 #pragma unroll
-                        for (int ks = 0; ks < DH / 16; ++ks) {
+                        for (int ks = 0; ks < C::KSTEPS; ++ks) {
                             const uint64_t qoff = (uint64_t)((((ks >> 2) * C::QCHUNK) + (ks & 3) * 32) >> 4);
                             const uint64_t koff = (uint64_t)((((ks >> 2) * C::CHUNK) + (ks & 3) * 32) >> 4);
-                            mma_ss(sd, qdesc + qoff, kdesc + koff, idS, ks > 0);
+                            if constexpr (F8)
+                                mma_ss_f8(sd, qdesc + qoff, kdesc + koff, idS, ks > 0);
+                            else
+                                mma_ss(sd, qdesc + qoff, kdesc + koff, idS, ks > 0);
                         }
                         TL(32, qt);
                         tc_commit(&sh.s_full[reg]);
@@ -374,7 +400,7 @@ __global__ void __launch_bounds__(512, 1)
             // reads only each item's first record; per tile it waits for P(t) and for the epilogue's
             // read of O(t-1), and commits one barrier (pv_done: region R[t % 3] free, O(t) ready)
             if (lane == 0) {
-                constexpr uint32_t idPV = idesc_bf16_f32(128, DH, true);
+                constexpr uint32_t idPV = F8 ? idesc_e4m3_f32(128, DH, true) : idesc_bf16_f32(128, DH, true);
                 const uint32_t aKV = smem_u32(sKV);
                 int qt = 0;
                 bool ok = true;
@@ -397,9 +423,15 @@ __global__ void __launch_bounds__(512, 1)
                         TL(12, qt);
                         tc_fence_after();
                         const uint32_t acol = tmem + a_col(qt);
+                        // one step = 32 bytes of keys: 16 (bf16) or 32 (E4M3) rows of V, 8 columns of P
 #pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) // 16 keys = 2048 bytes of V per step
-                            mma_ts(tmem + kOCol, acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
+                        for (int ks = 0; ks < 128 * C::EB / 32; ++ks) {
+                            if constexpr (F8)
+                                mma_ts_f8(tmem + kOCol, acol + ks * 8, vdesc + (uint64_t)(ks * 32 * DH / 16), idPV,
+                                          ks > 0);
+                            else
+                                mma_ts(tmem + kOCol, acol + ks * 8, vdesc + (uint64_t)(ks * 128), idPV, ks > 0);
+                        }
                         TL(36, qt);
                         tc_commit(&sh.pv_done[reg]);
                         if (t == rec.ntiles - 1) tc_commit(&sh.kv_empty[vb]); // the item's V is no longer read
@@ -429,9 +461,13 @@ __global__ void __launch_bounds__(512, 1)
             const TileRec rec = sh.rec[rs];
             if (rec.npos < 0) break;
             const int reg = qt % kRegions;
+            const int e_row = pl < rec.npos ? sh.rec_e[rs][pl] : 0;
             // last visible key column of this half (keys after the query are masked on the diagonal block)
-            const int limit =
-                (pl < rec.npos ? min(127, sh.rec_e[rs][pl] / a.k - rec.tok0) : 127) - 64 * beta;
+            const int limit = (pl < rec.npos ? min(127, e_row / a.k - rec.tok0) : 127) - 64 * beta;
+            float sq = 1.f; // FP8: the row's q scale
+            if constexpr (F8) {
+                if (pl < rec.npos) sq = a.qs[(int64_t)(rec.r * G + row % G) * a.sstride + e_row / a.k];
+            }
             if (!wait_or_abort(&sh.s_full[reg], (qt / kRegions) & 1, abort_flag, a.err, 26, kWaitLimit)) break;
             if (row == 0 && beta == 0) TL(4, qt);
             tc_fence_after();
@@ -441,6 +477,22 @@ __global__ void __launch_bounds__(512, 1)
             tmem_ld32_at<32>(sadr + 64 * beta + 32, s);
             tmem_ld_wait();
             if (row == 0 && beta == 0) TL(14, qt);
+            const int vbuf = (2 * rec.item + 1) % NKV; // FP8: the buffer of the item's V load and scales
+            if constexpr (F8) {
+                // logits in units of the codes: q8 . k8 * s_k (the row's s_q * scale enters the exponent)
+                if (!wait_or_abort(&sh.kv_full[vbuf], ((2 * rec.item + 1) / NKV) & 1, abort_flag, a.err, 45,
+                                   kWaitLimit))
+                    break;
+                const float4* ksc = reinterpret_cast<const float4*>(sh.fscl[vbuf][0] + 64 * beta);
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    const float4 k4 = ksc[c / 4];
+                    s[c] = __float_as_uint(__uint_as_float(s[c]) * k4.x);
+                    s[c + 1] = __float_as_uint(__uint_as_float(s[c + 1]) * k4.y);
+                    s[c + 2] = __float_as_uint(__uint_as_float(s[c + 2]) * k4.z);
+                    s[c + 3] = __float_as_uint(__uint_as_float(s[c + 3]) * k4.w);
+                }
+            }
             if (limit < 63) {
 #pragma unroll
                 for (int c = 0; c < 64; ++c)
@@ -461,9 +513,37 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
             if (row == 0 && beta == 0) TL(33, qt);
             const float m = fmaxf(sh.xmax[qt & 1][0][row], sh.xmax[qt & 1][1][row]);
-            const uint64_t sl2x2 = f2_pack(sl2, sl2);
-            const uint64_t nmx2 = f2_pack(-m * sl2, -m * sl2);
+            const float cl2 = F8 ? sl2 * sq : sl2; // logit -> log2 units
+            const uint64_t sl2x2 = f2_pack(cl2, cl2);
+            const uint64_t nmx2 = f2_pack(-m * cl2, -m * cl2);
             uint64_t l2 = 0, lr2 = 0;
+            if constexpr (F8) {
+                // P' = P * s_v * C_b (at most 448) rounded to E4M3 for the PV product; the row sum of the
+                // weights it stands for, P'_q / (s_v * C_b) = P'_q * (1 / s_v) / C_b, normalises O: the
+                // partial is O / sum(P'_q / s_v) (the C_b cancel), an exact weighted average of V rows
+                const float cb = sh.fcb[vbuf];
+                const float4* vsc = reinterpret_cast<const float4*>(sh.fscl[vbuf][1] + 64 * beta);
+                const float4* rvc = reinterpret_cast<const float4*>(sh.fscl[vbuf][2] + 64 * beta);
+                uint32_t pk[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int c = 4 * q;
+                    const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2x2, nmx2);
+                    const uint64_t x23 =
+                        f2_fma(f2_pack(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])), sl2x2, nmx2);
+                    const float e0 = ex2_approx(f2_lo(x01)), e1 = ex2_approx(f2_hi(x01));
+                    const float e2 = ex2_approx(f2_lo(x23)), e3 = ex2_approx(f2_hi(x23));
+                    l2 = f2_add(l2, f2_add(f2_pack(e0, e1), f2_pack(e2, e3)));
+                    const float4 v4 = vsc[q], r4 = rvc[q];
+                    const uint32_t w01 = e4m3x2_pack(e0 * v4.x * cb, e1 * v4.y * cb);
+                    const uint32_t w23 = e4m3x2_pack(e2 * v4.z * cb, e3 * v4.w * cb);
+                    pk[q] = w01 | (w23 << 16);
+                    const float2 d01 = e4m3x2_unpack(w01), d23 = e4m3x2_unpack(w23);
+                    lr2 = f2_fma(f2_pack(d01.x, d01.y), f2_pack(r4.x, r4.y), lr2);
+                    lr2 = f2_fma(f2_pack(d23.x, d23.y), f2_pack(r4.z, r4.w), lr2);
+                }
+                tmem_st16(sadr + 16 * beta, pk);
+            } else {
 #pragma unroll
             for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t pk[16];
@@ -479,10 +559,12 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 tmem_st16(sadr + 32 * beta + c4 * 16, pk);
             }
+            }
             // the exact sum gives the lse (the combine's merge weight); the sum of the bf16-rounded P
             // that the PV product uses normalises O, so each partial is an exact weighted average
             sh.lsum[qt & 3][beta][row] = make_float2(f2_lo(l2) + f2_hi(l2), f2_lo(lr2) + f2_hi(lr2));
-            if (beta == 0) sh.mrow[qt & 3][row] = m;
+            // row max: of the raw scores (bf16), of the logits in natural units (FP8)
+            if (beta == 0) sh.mrow[qt & 3][row] = F8 ? m * sq * (sl2 * 0.6931471805599453f) : m;
             if (row == 0 && beta == 0) TL(34, qt);
             tmem_st_wait();
             if (row == 0 && beta == 0) TL(35, qt);
@@ -519,7 +601,7 @@ __global__ void __launch_bounds__(512, 1)
             if (row == 0) TL(6, qt);
             tc_fence_after();
             const float2 la = sh.lsum[qt & 3][0][row], lb = sh.lsum[qt & 3][1][row];
-            const float lse_row = sh.mrow[qt & 3][row] * scale + logf(la.x + lb.x);
+            const float lse_row = (F8 ? sh.mrow[qt & 3][row] : sh.mrow[qt & 3][row] * scale) + logf(la.x + lb.x);
             const float inv_l = 1.f / (la.y + lb.y);
             const int h = rec.r * G + hh;
             const int64_t prow = (int64_t)(p - a.row0);
@@ -573,16 +655,17 @@ __global__ void __launch_bounds__(512, 1)
 #undef TL
 }
 
-template <int DH, int G>
+template <int DH, int G, bool F8>
 cudaError_t launch_cfg(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
                        cudaStream_t s, int n_sm)
 {
-    using C = AttnCfg<DH, G>;
+    using C = AttnCfg<DH, G, F8>;
     const int smem = C::SMEM + (int)sizeof(AttnShared);
     static_assert(C::SMEM + sizeof(AttnShared) <= 227 * 1024, "shared memory budget");
-    cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<DH, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(sparse_attn_kernel<DH, G, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    sparse_attn_kernel<DH, G><<<n_sm, 512, smem, s>>>(a, qmap, kmap, vmap);
+    sparse_attn_kernel<DH, G, F8><<<n_sm, 512, smem, s>>>(a, qmap, kmap, vmap);
     note_launch(1);
     return cudaGetLastError();
 }
@@ -592,19 +675,36 @@ cudaError_t launch_dh(const AttnArgs& a, int G, const CUtensorMap& qmap, const C
                       const CUtensorMap& vmap, cudaStream_t s, int n_sm)
 {
     switch (G) {
-    case 1: return launch_cfg<DH, 1>(a, qmap, kmap, vmap, s, n_sm);
-    case 2: return launch_cfg<DH, 2>(a, qmap, kmap, vmap, s, n_sm);
-    case 4: return launch_cfg<DH, 4>(a, qmap, kmap, vmap, s, n_sm);
-    case 8: return launch_cfg<DH, 8>(a, qmap, kmap, vmap, s, n_sm);
-    case 16: return launch_cfg<DH, 16>(a, qmap, kmap, vmap, s, n_sm);
-    case 32: return launch_cfg<DH, 32>(a, qmap, kmap, vmap, s, n_sm);
-    case 64: return launch_cfg<DH, 64>(a, qmap, kmap, vmap, s, n_sm);
-    case 128: return launch_cfg<DH, 128>(a, qmap, kmap, vmap, s, n_sm);
+    case 1: return launch_cfg<DH, 1, false>(a, qmap, kmap, vmap, s, n_sm);
+    case 2: return launch_cfg<DH, 2, false>(a, qmap, kmap, vmap, s, n_sm);
+    case 4: return launch_cfg<DH, 4, false>(a, qmap, kmap, vmap, s, n_sm);
+    case 8: return launch_cfg<DH, 8, false>(a, qmap, kmap, vmap, s, n_sm);
+    case 16: return launch_cfg<DH, 16, false>(a, qmap, kmap, vmap, s, n_sm);
+    case 32: return launch_cfg<DH, 32, false>(a, qmap, kmap, vmap, s, n_sm);
+    case 64: return launch_cfg<DH, 64, false>(a, qmap, kmap, vmap, s, n_sm);
+    case 128: return launch_cfg<DH, 128, false>(a, qmap, kmap, vmap, s, n_sm);
     default: return cudaErrorInvalidValue;
     }
 }
 
 } // namespace
+
+cudaError_t launch_sparse_attn_fp8(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                                   const CUtensorMap& vmap, cudaStream_t s)
+{
+    int dev = 0, n_sm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (a.d_h != 128) return cudaErrorInvalidValue;
+    switch (a.H_q / a.H_kv) {
+    case 1: return launch_cfg<128, 1, true>(a, qmap, kmap, vmap, s, n_sm);
+    case 2: return launch_cfg<128, 2, true>(a, qmap, kmap, vmap, s, n_sm);
+    case 4: return launch_cfg<128, 4, true>(a, qmap, kmap, vmap, s, n_sm);
+    case 8: return launch_cfg<128, 8, true>(a, qmap, kmap, vmap, s, n_sm);
+    case 16: return launch_cfg<128, 16, true>(a, qmap, kmap, vmap, s, n_sm);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                                const CUtensorMap& vmap, cudaStream_t s)

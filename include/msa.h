@@ -10,6 +10,8 @@
  *          chunking, two-stage forward with an LSE split-K combine, LSE emitted for the backward).
  *   [ABS]  The paper abstract ("MiniMax Sparse Attention", arXiv 2606.13392): Top-k per GQA
  *          group, exact block-sparse attention over the selected blocks, prefill and decoding.
+ *   [BLOG] The "MiniMax M3" sparse-attention blog post, kernel paragraph: the attention kernels
+ *          were tuned on FP8 tensor cores.
  *
  * Conventions shared by every entry point
  *   - bf16 tensors are passed as uint16_t bit patterns (msa_bf16).
@@ -210,6 +212,43 @@ MSA_API msa_status msa_sparse_prefill(const msa_bf16* q, const msa_bf16* k, cons
                               int d_h, int B_k, int kk, const int32_t* block_idx, const msa_kv2q_layout* layout,
                               const void* kv2q, msa_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
                               msa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * FP8 main branch                               [BLOG: kernel paragraph, FP8 tensor cores]
+ *
+ * The page names FP8 tensor cores for the attention kernels and gives no quantisation; reading:
+ * q, k and v are quantised row by row, one scale per (token, head) row, to OCP E4M3 (bias 7,
+ * subnormals, largest finite 448, no infinities): scale = amax / 448 (1 for an all-zero row),
+ * code = nearest E4M3 value of x / scale (ties to the even code, |x / scale| >= 448 saturates).
+ * The main branch is then the exact attention of msa_sparse_prefill on the dequantised values
+ * code * scale.
+ *
+ * msa_quantize_e4m3: x [N, H, d] bf16 (d in {64, 128}) ->
+ *   codes   : [N, H, d] uint8 E4M3 codes (the quotient x / scale is formed in fp64, so codes are
+ *             bit-identical to the definition above)
+ *   scales  : [H, S] fp32, S = N rounded up to a multiple of 128 (head-major; tokens N..S-1 get 1)
+ *   rscales : [H, S] fp32 = 1 / scales, or NULL
+ *   blkmax  : [H, S / 128] fp32 = largest scale of each 128-token block, or NULL (cleared here)
+ * All device pointers 16-byte aligned (blkmax 4). Asynchronous on `stream`, no workspace.
+ *
+ * msa_sparse_prefill_fp8: the main branch on E4M3 inputs (d_h = 128, G <= 16): q8, qs from
+ * msa_quantize_e4m3 of q; k8, ks of k; v8, vs, rvs, vblkmax of v (all three outputs). The S = QK^T
+ * and PV products run on the FP8 tensor cores (tcgen05 kind::f8f6f4) with fp32 accumulation; the
+ * k scales enter the logits per key, the q scale per row; the attention weights P are scaled by
+ * the key's v scale and 448 / (the block's largest v scale) and rounded to E4M3 for the PV product,
+ * and each partial output is normalised by the sum of the weights those codes stand for (so it is
+ * an exact weighted average of V rows); the lse uses the unrounded weights. Arguments, layout,
+ * workspace (msa_sparse_prefill_workspace_size) and outputs as for msa_sparse_prefill.
+ * ------------------------------------------------------------------------------------------ */
+MSA_API msa_status msa_quantize_e4m3(const msa_bf16* x, int64_t N, int H, int d, uint8_t* codes, float* scales,
+                                     float* rscales, float* blkmax, msa_stream_t stream);
+
+MSA_API msa_status msa_sparse_prefill_fp8(const uint8_t* q8, const float* qs, const uint8_t* k8, const float* ks,
+                                          const uint8_t* v8, const float* vs, const float* rvs, const float* vblkmax,
+                                          int64_t N, int H_q, int H_kv, int d_h, int B_k, int k,
+                                          const int32_t* block_idx, const msa_kv2q_layout* layout, const void* kv2q,
+                                          msa_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
+                                          msa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
  * Backward: main-branch gradients (selections fixed) and the index-branch KL signal [EXPL 03, 05]

@@ -730,6 +730,8 @@ uint8_t msa_oracle_e4m3_encode(double x)
 int msa_oracle_quantize_e4m3_rows(const uint16_t* x, int64_t rows, int cols, uint8_t* codes, double* scales)
 {
     if (!x || !codes || !scales || rows < 0 || cols < 1) return -1;
+    /* rows are independent: one row per iteration, any thread */
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         double amax = 0.0;
         for (int c = 0; c < cols; ++c) {
