@@ -46,6 +46,7 @@ def parse_args():
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch (varlen) prefill leg")
     ap.add_argument("--no-backward", action="store_true", help="skip the main-branch backward leg")
     ap.add_argument("--no-long", action="store_true", help="skip the 1M-token prefill leg")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 main-branch leg")
     ap.add_argument("--decode-workload", default=synth.DECODE64.name, choices=sorted(synth.DECODE_CONFIGS))
     ap.add_argument("--e2e-steps", type=int, default=8,
                     help="pipelined host-buffer steps (the first input copy and the last output copy are not overlapped)")
@@ -498,6 +499,49 @@ def gpu_arm(args, rank, world):
                   "note": "msa_sparse_prefill_varlen: index branch, inversion, attention and combine in one call"}
         del vt, v_out, v_lse, v_bi, v_ws
 
+    # FP8 main branch on the same workload and selections: E4M3 quantisation of q, k, v (timed, part of
+    # the step) and the attention on FP8 tensor cores + combine; index branch and inversion as above
+    fp8 = None
+    if not args.no_fp8 and d_h == 128:
+        f_out = torch.empty_like(out)
+        f_lse = torch.empty_like(lse)
+
+        def fp8_step():
+            qq, kq, vq = (msa.msa_quantize_e4m3(t[n]) for n in ("q", "k", "v"))
+            msa.msa_sparse_prefill_fp8(qq, kq, vq, block_idx, kv, out=f_out, lse=f_lse, workspace=ws_pf)
+
+        for _ in range(args.warmup):
+            fp8_step()
+        torch.cuda.synchronize()
+        if msa.msa_get_device_error(ws_pf) != 0:
+            raise RuntimeError("device error in the FP8 warm-up")
+        fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        ftrace = msa.KernelTrace(16 * args.steps)
+        with ftrace:
+            for st in range(args.steps):
+                flush.zero_()
+                fev[st][0].record()
+                fp8_step()
+                fev[st][1].record()
+        torch.cuda.synchronize()
+        (f_ms,) = replicas.max_over_ranks([sum(a.elapsed_time(b) for a, b in fev)], device=dev)
+        fk = {n: sum(d) / args.steps for n, d in ftrace.durations().items()}
+        peak8 = 2.0 * peaks["bf16_tflops"]
+        ach8 = roofline.main_branch_flops(N, H_q, d_h, k, cfg.B_k) / (fk["attn"] / 1000.0) / 1e12
+        qb = (roofline.quant_bytes(N, H_q, d_h) + 2 * roofline.quant_bytes(N, H_kv, d_h))
+        fp8 = {"ms_per_step": f_ms / args.steps, "kernels_ms": fk,
+               "roofline": {"kernel": "attn (fp8)", "bound": "tensor", "achieved": ach8, "unit": "TFLOP/s",
+                            "peak": peak8, "frac": ach8 / peak8,
+                            "peak_source": "measured bf16 burst x 2 (nominal FP8 / bf16 dense ratio)"},
+               "quant": {"achieved": qb / (fk["quant"] / 1000.0) / 1e9, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                         "frac": qb / (fk["quant"] / 1000.0) / 1e9 / peaks["hbm_gbs"], "algorithmic": qb},
+               "prefill_tokens_per_s": replicas.aggregate_rate(
+                   N * args.steps, world,
+                   (f_ms + sum(sum(kern.get(n, [0.0])) for n in ("index_topk", "kv2q"))) / 1000.0),
+               "note": "E4M3 quantisation of q, k, v + FP8 attention + combine per step; prefill_tokens_per_s "
+                       "adds the bf16 index branch and inversion times of the main leg"}
+        del f_out, f_lse
+
     # main-branch backward on the same workload, selections held fixed: gradients of sum(dout * out) in
     # q, k, v from the forward's out and lse of the timed steps
     backward = None
@@ -628,7 +672,7 @@ def gpu_arm(args, rank, world):
                         "ms_per_step": dec_total / args.steps} if dcfg else None),
             "decode_graph": decode_graph,
             "roofline": roof, "kernels": kstats, "cpu_baseline": cpu_base, "e2e": e2e, "varlen": varlen,
-            "backward": backward, "long_prefill": long_prefill,
+            "backward": backward, "long_prefill": long_prefill, "fp8": fp8,
             "gpu_launches": int(launches), "clocks": clocks.summary(), "wall_s_timed": wall}
     print(json.dumps(line), flush=True)
 

@@ -72,7 +72,7 @@ SIGNATURES = [
 ]
 
 KERNEL_NAMES = {1: "index_topk", 2: "kv2q", 3: "attn", 4: "combine", 5: "dec_pool", 6: "dec_topk", 7: "dec_attn",
-                8: "dec_combine", 9: "bwd_prep", 10: "bwd_attn", 11: "bwd_convert"}
+                8: "dec_combine", 9: "bwd_prep", 10: "bwd_attn", 11: "bwd_convert", 12: "quant"}
 
 
 class msa_trace(ctypes.Structure):

@@ -3,14 +3,15 @@
 // (token, head) row, scale = amax / 448, codes rounded to nearest with ties to the even code,
 // saturating at 448, subnormals kept).
 //
-// One warp per row of d_h elements: the row's amax by warp shuffles, then every element's code from
-// its quotient x / scale computed in fp64 exactly as the definition states (two correctly rounded
-// fp64 divisions), so the rounding decision at a code midpoint is the same on every conforming
-// implementation. Besides the codes the kernel writes the row scales and their reciprocals in a
-// head-major layout [H][S] (S = N rounded up to whole 128-token blocks, padding tokens get scale 1 so
+// One warp per row of d_h elements: the row's amax by warp shuffles, then every element's code. The
+// code is decided in fp32 with the hardware E4M3 conversion when the fp32 quotient is clearly away
+// from a code midpoint, and otherwise from the quotient x / scale computed in fp64 exactly as the
+// definition states (two correctly rounded fp64 divisions), so every code equals the definition's.
+// Besides the codes the kernel writes the row scales and their reciprocals in a head-major layout [H][S] (S = N rounded up to whole 128-token blocks, padding tokens get scale 1 so
 // that every block's scale run is finite and 512 bytes long), and optionally the largest scale of
 // every (head, 128-token block), which the attention uses to keep the FP8 P' = P * s_v in range.
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace msa {
 
@@ -35,6 +36,26 @@ __device__ __forceinline__ uint8_t e4m3_encode_rne(double q)
     return sign | (uint8_t)(((E + 7) << 3) | (n - 8));
 }
 
+// Code of x / scale with r = 448 / amax in fp32: the fp32 quotient x * r is within 2^-23 (relative)
+// of the exact one, i.e. within 2 units of the 20 mantissa bits E4M3 drops; unless it lies within 8
+// such units of a code midpoint (or of a subnormal-step midpoint), the hardware conversion (round to
+// nearest even, saturating) gives the exact code; otherwise the fp64 quotient decides.
+__device__ __forceinline__ uint8_t e4m3_code(float x, float r, double scale)
+{
+    const float q = x * r;
+    const float a = fabsf(q);
+    bool near;
+    if (a >= 0.015625f) {
+        const uint32_t rem = __float_as_uint(a) & 0xFFFFFu;
+        near = rem > 0x80000u - 8u && rem < 0x80000u + 8u;
+    } else {
+        const float t = a * 512.f; // exact: the subnormal grid in units of 2^-9
+        near = fabsf(t - floorf(t) - 0.5f) < 1.0e-4f;
+    }
+    if (near) return e4m3_encode_rne((double)x / scale);
+    return (uint8_t)(e4m3x2_pack(q, 0.f) & 0xFFu);
+}
+
 __global__ void quantize_e4m3_kernel(QuantArgs a)
 {
     const int lane = threadIdx.x & 31;
@@ -50,21 +71,32 @@ __global__ void quantize_e4m3_kernel(QuantArgs a)
         float amax = 0.f;
         if (row < nrows) {
             const uint16_t* src = a.x + row * a.d + lane * per;
+            if (per == 4) { // one 8-byte load per lane (the row is 256 bytes, 16-byte aligned)
+                const uint2 v = *reinterpret_cast<const uint2*>(src);
+                x[0] = bf16_lo(v.x), x[1] = bf16_hi(v.x), x[2] = bf16_lo(v.y), x[3] = bf16_hi(v.y);
+            } else {
+#pragma unroll
+                for (int i = 0; i < kMaxPer; ++i)
+                    if (i < per) x[i] = __uint_as_float((uint32_t)src[i] << 16);
+            }
 #pragma unroll
             for (int i = 0; i < kMaxPer; ++i)
-                if (i < per) {
-                    x[i] = __uint_as_float((uint32_t)src[i] << 16);
-                    amax = fmaxf(amax, fabsf(x[i]));
-                }
+                if (i < per) amax = fmaxf(amax, fabsf(x[i]));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const double scale = amax > 0.f ? (double)amax / 448.0 : 1.0;
+        const float r = (float)(1.0 / scale);
         if (row < nrows) {
             uint8_t* dst = a.codes + row * a.d + lane * per;
+            uint8_t c[kMaxPer];
 #pragma unroll
             for (int i = 0; i < kMaxPer; ++i)
-                if (i < per) dst[i] = e4m3_encode_rne((double)x[i] / scale);
+                if (i < per) c[i] = e4m3_code(x[i], r, scale);
+            if (per == 4)
+                *reinterpret_cast<uint32_t*>(dst) = c[0] | (c[1] << 8) | (c[2] << 16) | ((uint32_t)c[3] << 24);
+            else
+                for (int i = 0; i < per; ++i) dst[i] = c[i];
         }
         if (lane == 0) {
             const float s32 = (float)scale;

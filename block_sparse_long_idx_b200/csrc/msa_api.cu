@@ -85,6 +85,19 @@ constexpr size_t kErrBytes = 256;
 constexpr int kDefaultWindow = 2048;
 constexpr int kDefaultChunk = 512;
 
+// Default query window: N / 128 rounded up to a power of two within [2048, 16384] for one sequence
+// (nb = ceil(N / 128)), 2048 for a packed batch. A window's rows select about W * (k - 1) / (visible
+// blocks) rows per (window, block) item, ~30 at mid-sequence with W = N / 128, so the 128-row tiles of
+// an item stay nearly full on long sequences, while short ones keep small windows whose gathered
+// query rows stay in L2.
+int default_window(int64_t N, int64_t nb)
+{
+    if (nb != (N + kBk - 1) / kBk) return kDefaultWindow; // packed batch of sequences
+    int w = kDefaultWindow;
+    while (w < 16384 && (int64_t)w < N / kBk) w *= 2;
+    return w;
+}
+
 size_t kv2q_internal_tmp(const msa_kv2q_layout& L)
 {
     return kv2q_scan_tmp_bytes((int64_t)L.H_kv * L.nb * L.n_windows, L.H_kv);
@@ -222,7 +235,7 @@ static msa_status layout_fill(int64_t N, int H_kv, int B_k, int k, int64_t nb, i
 {
     if (!L || N < 1 || H_kv < 1 || B_k < 1 || k < 1 || window < 0 || chunk < 0 || nb < 1) return MSA_ERR_INVALID_ARG;
     if (B_k != kBk || k > kMaxK || N > kMaxN || nb > (int64_t)kMaxN) return MSA_ERR_UNSUPPORTED;
-    if (window == 0) window = kDefaultWindow;
+    if (window == 0) window = default_window(N, nb);
     if (chunk == 0) chunk = kDefaultChunk < window ? kDefaultChunk : window;
     if (window % kBk != 0 || chunk > window) return MSA_ERR_INVALID_ARG;
     memset(L, 0, sizeof *L);
@@ -528,7 +541,10 @@ msa_status msa_quantize_e4m3(const msa_bf16* x, int64_t N, int H, int d, uint8_t
     if (blkmax)
         if (msa_status st = cuda_status(cudaMemsetAsync(blkmax, 0, (size_t)H * a.nb * 4, s), "clearing blkmax"))
             return st;
-    return cuda_status(launch_quantize_e4m3(a, s), "quantize launch");
+    trace_begin(s);
+    const cudaError_t e = launch_quantize_e4m3(a, s);
+    trace_end(s, MSA_KERNEL_QUANT);
+    return cuda_status(e, "quantize launch");
 }
 
 msa_status msa_sparse_prefill_fp8(const uint8_t* q8, const float* qs, const uint8_t* k8, const float* ks,

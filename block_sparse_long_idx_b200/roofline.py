@@ -81,3 +81,10 @@ def kv2q_bytes(N: int, H_kv: int, k: int, B_k: int, window: int = 2048) -> float
     slots = H_kv * N * k
     valid = n_selected(N, k, B_k) * H_kv
     return 8.0 * slots + 4.0 * valid + 12.0 * H_kv * nb * n_windows
+
+
+def quant_bytes(N: int, H: int, d: int, B_k: int = 128) -> float:
+    """E4M3 quantisation of one [N, H, d] bf16 tensor: read 2 B and write a 1-byte code per element, write
+    the scale and its reciprocal (4 B each) per row of the padded token range and the block maxima."""
+    S = (N + B_k - 1) // B_k * B_k
+    return 3.0 * N * H * d + 8.0 * S * H + 4.0 * H * (S // B_k)

@@ -134,7 +134,9 @@ MSA_API msa_status msa_index_topk(const msa_bf16* q_idx, const msa_bf16* k_idx, 
  *                                      covers at most `chunk` consecutive entries of one list.
  *   window_items int32 [n_windows + 1] first item of each window; the last value is the count
  *   (plus internal per-(r, b, window) counts used while building)
- * window = 0 / chunk = 0 select the defaults (2048 rows per window, items of at most 512 entries).
+ * window = 0 / chunk = 0 select the defaults: windows of N / 128 rows rounded up to a power of two
+ * within [2048, 16384] (2048 up to N = 256K; longer sequences get longer windows so that each
+ * (window, block) item keeps its 128-row tiles nearly full), items of at most 512 entries.
  * ------------------------------------------------------------------------------------------ */
 typedef struct {
     int32_t r;     /* GQA group */
@@ -386,7 +388,8 @@ typedef enum {
     MSA_KERNEL_DEC_COMBINE = 8, /* decode LSE combine                                           */
     MSA_KERNEL_BWD_PREP = 9,    /* backward: rowsum(dout * out)                                 */
     MSA_KERNEL_BWD_ATTN = 10,   /* backward: KV-outer gradients                                 */
-    MSA_KERNEL_BWD_CONVERT = 11 /* backward: fp32 accumulators to bf16                          */
+    MSA_KERNEL_BWD_CONVERT = 11, /* backward: fp32 accumulators to bf16                         */
+    MSA_KERNEL_QUANT = 12       /* E4M3 quantisation of one tensor                               */
 } msa_kernel_id;
 
 typedef struct {
