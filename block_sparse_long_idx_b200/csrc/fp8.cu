@@ -39,11 +39,14 @@ __device__ __forceinline__ uint8_t e4m3_encode_rne(double q)
 // Code of x / scale with r = 448 / amax in fp32: the fp32 quotient x * r is within 2^-23 (relative)
 // of the exact one, i.e. within 2 units of the 20 mantissa bits E4M3 drops; unless it lies within 8
 // such units of a code midpoint (or of a subnormal-step midpoint), the hardware conversion (round to
-// nearest even, saturating) gives the exact code; otherwise the fp64 quotient decides.
-__device__ __forceinline__ uint8_t e4m3_code(float x, float r, double scale)
+// nearest even, saturating) gives the exact code; otherwise the fp64 quotient x / (amax / 448), the
+// definition's, decides.
+__device__ __forceinline__ uint8_t e4m3_code(float x, float r, float amax)
 {
     const float q = x * r;
     const float a = fabsf(q);
+    if (!(r < 3.0e38f)) // amax below ~1.3e-36: 448 / amax overflows fp32, the fp64 quotient is finite
+        return e4m3_encode_rne((double)x / ((double)amax / 448.0));
     bool near;
     if (a >= 0.015625f) {
         const uint32_t rem = __float_as_uint(a) & 0xFFFFFu;
@@ -52,7 +55,7 @@ __device__ __forceinline__ uint8_t e4m3_code(float x, float r, double scale)
         const float t = a * 512.f; // exact: the subnormal grid in units of 2^-9
         near = fabsf(t - floorf(t) - 0.5f) < 1.0e-4f;
     }
-    if (near) return e4m3_encode_rne((double)x / scale);
+    if (near) return e4m3_encode_rne((double)x / ((double)amax / 448.0));
     return (uint8_t)(e4m3x2_pack(q, 0.f) & 0xFFu);
 }
 
@@ -65,8 +68,8 @@ __global__ void quantize_e4m3_kernel(QuantArgs a)
     constexpr int kMaxPer = 8; // d <= 256
     const int per = a.d / 32;
     for (int64_t row = warp0; row < a.N_pad * a.H; row += nwarps) {
-        const int64_t n = row / a.H;
-        const int h = (int)(row - n * a.H);
+        const int n = (int)((uint32_t)row / (uint32_t)a.H); // N_pad * H < 2^31
+        const int h = (int)(row - (int64_t)n * a.H);
         float x[kMaxPer];
         float amax = 0.f;
         if (row < nrows) {
@@ -85,23 +88,25 @@ __global__ void quantize_e4m3_kernel(QuantArgs a)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const double scale = amax > 0.f ? (double)amax / 448.0 : 1.0;
-        const float r = (float)(1.0 / scale);
+        // fp32 divisions, correctly rounded: for a bf16 amax neither amax / 448 nor 448 / amax lies within
+        // 2^-53 (relative) of an fp32 rounding midpoint (448 = 7 * 2^6), so these equal the fp32
+        // roundings of the definition's fp64 scale and of its reciprocal
+        const float s32 = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+        const float r = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
         if (row < nrows) {
             uint8_t* dst = a.codes + row * a.d + lane * per;
             uint8_t c[kMaxPer];
 #pragma unroll
             for (int i = 0; i < kMaxPer; ++i)
-                if (i < per) c[i] = e4m3_code(x[i], r, scale);
+                if (i < per) c[i] = e4m3_code(x[i], r, amax);
             if (per == 4)
                 *reinterpret_cast<uint32_t*>(dst) = c[0] | (c[1] << 8) | (c[2] << 16) | ((uint32_t)c[3] << 24);
             else
                 for (int i = 0; i < per; ++i) dst[i] = c[i];
         }
         if (lane == 0) {
-            const float s32 = (float)scale;
             a.scales[(int64_t)h * a.N_pad + n] = s32;
-            if (a.rscales) a.rscales[(int64_t)h * a.N_pad + n] = (float)(1.0 / scale);
+            if (a.rscales) a.rscales[(int64_t)h * a.N_pad + n] = r;
             // scales are positive: their bit patterns order like the values
             if (a.blkmax && row < nrows)
                 atomicMax(reinterpret_cast<int*>(a.blkmax) + (int64_t)h * a.nb + n / kBk, __float_as_int(s32));

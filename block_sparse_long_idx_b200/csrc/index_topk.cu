@@ -8,9 +8,12 @@
 // that owns TMEM lane i reads its row's 128 scores, max-pools them, and offers the pooled score to
 // its register Top-k list. The pooled score matrix never leaves the SM.
 //
-// Roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner),
-// warps 4-7 = epilogue of tile tA, warps 8-11 = epilogue of tile tB. Persistent CTAs walk items in
-// decreasing work order with a boustrophedon assignment.
+// Roles (384 threads): warp 0 = TMA producer, warps 1 and 2 = MMA issuers of tiles tA and tB (warp 1
+// also owns TMEM), warps 4-7 = epilogue of tile tA, warps 8-11 = epilogue of tile tB. A thread
+// stays busy about as long as the tensor pipe takes to run the MMAs it issues, plus tens of cycles
+// per barrier wait and commit, so each tile has its own issuer and the barriers the two share
+// (k_idx stage free, accumulator full, query tiles free) take one arrival from each. Persistent
+// CTAs walk items in decreasing work order with a boustrophedon assignment.
 #include <cstdio>
 
 #include "common.cuh"
@@ -104,14 +107,14 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&sh.q_full, 1);
-        mbar_init(&sh.q_empty, 1);
-        mbar_init(&sh.done, 1);
+        mbar_init(&sh.q_empty, 2);
+        mbar_init(&sh.done, 2);
         for (int s = 0; s < C::NST; ++s) {
             mbar_init(&sh.kv_full[s], 1);
-            mbar_init(&sh.kv_empty[s], 1);
+            mbar_init(&sh.kv_empty[s], 2);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sh.acc_full[b], 1);
+            mbar_init(&sh.acc_full[b], 2);
             mbar_init(&sh.acc_empty[b], 8);
         }
         sh.abort_flag = 0;
@@ -164,8 +167,9 @@ __global__ void __launch_bounds__(384, 1)
                 drain_wait(&sh.kv_full[g % C::NST], (g / C::NST) & 1, a.err, 7, kWaitLimit);
             if (item_cnt > 0) drain_wait(&sh.q_full, (item_cnt - 1) & 1, a.err, 8, kWaitLimit);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------------------------ MMA issuers (warp 1: tile A, 2: tile B)
+        const int tsel = warp - 1;
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
             const uint32_t aA = smem_u32(sqA), aB = smem_u32(sqB), ak = smem_u32(sk);
@@ -189,13 +193,17 @@ __global__ void __launch_bounds__(384, 1)
                     }
                     tc_fence_after();
                     const uint32_t kb = ak + s * C::TILE_BYTES;
+                    // tile A sees blocks 0 .. tA-1, tile B (when present) blocks 0 .. tA
+                    const bool mine = tsel == 0 ? b < itm.tA : tbv;
+                    if (mine) {
 #pragma unroll
-                    for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                        const int col = ks * 16;
-                        const uint32_t off = (col / C::CHUNK_COLS) * C::CHUNK_BYTES + (col % C::CHUNK_COLS) * 2;
-                        const uint64_t kd = desc_kmajor(kb + off, C::SWB);
-                        if (b < itm.tA) mma_ss(tmem + buf * 128, desc_kmajor(aA + off, C::SWB), kd, idesc, ks > 0);
-                        if (tbv) mma_ss(tmem + 256 + buf * 128, desc_kmajor(aB + off, C::SWB), kd, idesc, ks > 0);
+                        for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                            const int col = ks * 16;
+                            const uint32_t off = (col / C::CHUNK_COLS) * C::CHUNK_BYTES + (col % C::CHUNK_COLS) * 2;
+                            const uint64_t kd = desc_kmajor(kb + off, C::SWB);
+                            mma_ss(tmem + tsel * 256 + buf * 128, desc_kmajor((tsel ? aB : aA) + off, C::SWB), kd,
+                                   idesc, ks > 0);
+                        }
                     }
                     tc_commit(&sh.kv_empty[s]);
                     tc_commit(&sh.acc_full[buf]);

@@ -86,6 +86,8 @@ def test_quantize_e4m3_bit_exact():
                            3.49, -3.5], dtype=np.float32)
     x[7, 0, :] = synth.f32_to_bf16_bits(row)
     x[8, 3, :] = synth.f32_to_bf16_bits(rng.standard_normal(d).astype(np.float32) * 1e-3)  # small amax
+    # amax below 448 * FLT_MIN: 448 / amax overflows fp32, the definition's fp64 quotient does not
+    x[9, 0, :] = synth.f32_to_bf16_bits(rng.standard_normal(d).astype(np.float32) * np.float32(1e-37))
     xd = dev(x)
     q = msa.msa_quantize_e4m3(xd)
     torch.cuda.synchronize()
