@@ -67,13 +67,16 @@ def load_peaks():
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu capture of a smaller case of
 # the same kernel, per query row of the launch; partial outputs grow in proportion to the rows, so a
-# full launch is the per-row figure times its rows. A figure only applies to the sources it was
-# measured on: after any change to them the bench reports traffic as null.
+# full launch is the per-row figure times its rows. A figure only applies to the kernel source it was
+# measured on (the kernel's own .cu file, by hash): after any change to it the bench reports null.
 PROFILED_TRAFFIC = {
-    "attn": {"files": ("sparse_attn.cu", "common.cuh", "sm100.cuh"), "sha256_16": "94f46dc3167c3d8e",
-             "bytes_per_row": 308058.5,
-             "capture": "ncu capture of sparse_attn_kernel<128, 16> on the N=32768 prefill, one 8192-row pass"},
-    "combine": {"files": ("combine.cu", "common.cuh", "sm100.cuh"), "sha256_16": "efedf33b948eb033",
+    "attn": {"files": ("sparse_attn.cu",), "sha256_16": "cd81b9df8683b0b0",
+             "bytes_per_row": (382.179072e6 + 2.123139e9) / 8192,
+             "capture": "ncu capture of sparse_attn_kernel<128, 16, 0> on the N=32768 prefill, one 8192-row pass"},
+    "attn_fp8": {"files": ("sparse_attn.cu",), "sha256_16": "cd81b9df8683b0b0",
+                 "bytes_per_row": (224.727808e6 + 2.123034e9) / 8192,
+                 "capture": "ncu capture of sparse_attn_kernel<128, 16, 1> on the N=32768 prefill, one 8192-row pass"},
+    "combine": {"files": ("combine.cu",), "sha256_16": "8436940a71c651a1",
                 "bytes_per_row": 282506.7,
                 "capture": "ncu capture of combine_kernel on the N=32768 prefill, one 8192-row pass"},
 }
@@ -532,7 +535,9 @@ def gpu_arm(args, rank, world):
         fp8 = {"ms_per_step": f_ms / args.steps, "kernels_ms": fk,
                "roofline": {"kernel": "attn (fp8)", "bound": "tensor", "achieved": ach8, "unit": "TFLOP/s",
                             "peak": peak8, "frac": ach8 / peak8,
-                            "peak_source": "measured bf16 burst x 2 (nominal FP8 / bf16 dense ratio)"},
+                            "peak_source": "measured bf16 burst x 2 (nominal FP8 / bf16 dense ratio)",
+                            "traffic": profiled_traffic("attn_fp8", N), "traffic_source":
+                                PROFILED_TRAFFIC["attn_fp8"]["capture"] + ", scaled by rows per launch"},
                "quant": {"achieved": qb / (fk["quant"] / 1000.0) / 1e9, "unit": "GB/s", "peak": peaks["hbm_gbs"],
                          "frac": qb / (fk["quant"] / 1000.0) / 1e9 / peaks["hbm_gbs"], "algorithmic": qb},
                "prefill_tokens_per_s": replicas.aggregate_rate(
