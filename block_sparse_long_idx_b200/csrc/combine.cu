@@ -8,7 +8,7 @@
 //   out[i, h] = sum_s (w_s / L) * o_s,        lse[i, h] = M + log(L)
 // Slots are merged in the fixed order 0..n_sel-1, so the result is deterministic.
 //
-// Partials are laid out [row][slot][d_h/8][H_q][8] (bf16) and [row][slot][H_q] (fp32 lse). One CTA
+// Partials are laid out [row][slot][d_h/16][H_q][16] (bf16) and [row][slot][H_q] (fp32 lse). One CTA
 // per row reads the row's contiguous slabs with 16-byte loads (all slots of a unit in flight at
 // once), and stages the merged row in shared memory so the output row is written contiguously.
 #include <math_constants.h>
@@ -50,7 +50,9 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
     const int units = a.H_q * NC; // per slot
     const uint4* op = reinterpret_cast<const uint4*>(a.o_part + prow * a.k * a.H_q * (int64_t)a.d_h);
     for (int u = threadIdx.x; u < units; u += blockDim.x) {
-        const int c = u / a.H_q, h = u - c * a.H_q;
+        // 16-byte unit u of a slot in memory order: 32-byte unit u / (2 H_q), head (u / 2) % H_q, half u % 2
+        const int c2 = u / (2 * a.H_q), rem = u - c2 * 2 * a.H_q;
+        const int h = rem >> 1, c = 2 * c2 + (rem & 1);
         uint4 v[kMaxK];
 #pragma unroll
         for (int s = 0; s < kMaxK; ++s)

@@ -97,7 +97,7 @@ struct AttnArgs {
                                        // (differs from blk_tok when keys and queries are packed apart)
     long long* timeline;        // optional: CTA 0 records clock64 per tile event (nullptr = off)
     int timeline_tiles;         // capacity in tiles (48 event slots per tile)
-    uint16_t* o_part;           // [rows][k][d_h / 8][H_q][8] bf16 (normalised partial outputs)
+    uint16_t* o_part;           // [rows][k][d_h / 16][H_q][16] bf16 (normalised partial outputs)
     float* lse_part;            // [rows][k][H_q]
     int* err;
     // FP8 main branch (the q, k, v maps then hold E4M3 codes): head-major row scales [H][sstride]

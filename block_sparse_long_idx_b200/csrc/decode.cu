@@ -380,9 +380,9 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
         }
         const float inv = 1.f / lr;
         const int h = r * G + row;
-        // partial layout [sequence][slot][d_h/8][H_q][8] (as prefill's stage 1)
+        // partial layout [sequence][slot][d_h/16][H_q][16] (as prefill's stage 1)
         uint32_t* dst = reinterpret_cast<uint32_t*>(a.o_part + ((int64_t)beta * a.k + slot) * a.H_q * DH +
-                                                    ((int64_t)(col >> 3) * a.H_q + h) * 8 + (col & 7));
+                                                    ((int64_t)(col >> 4) * a.H_q + h) * 16 + (col & 15));
         *dst = pack_bf16x2(o0 * inv, o1 * inv);
         if (col == 0) {
             float Mr = -CUDART_INF_F;

@@ -315,6 +315,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
+// 32-byte global store of w[0..7] (the address must be 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(uint32_t* p, const uint32_t* w)
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
 // The two bf16 halves of a packed pair widened to fp32 (exact): low half, high half.
 __device__ __forceinline__ float bf16_lo(uint32_t pk) { return __uint_as_float(pk << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t pk) { return __uint_as_float(pk & 0xffff0000u); }

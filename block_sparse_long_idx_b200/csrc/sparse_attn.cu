@@ -610,9 +610,10 @@ __global__ void __launch_bounds__(512, 1)
                 report_error(a.err, MSA_ERR_DEVICE_CHECK, 300); // entry outside this pass: skip it
                 store = false;
             }
-            // partial layout [row][slot][d_h/8][H_q][8]: the G heads of a position are adjacent
-            // 16-byte units, so each warp-wide store writes contiguous runs
-            uint4* d4 = reinterpret_cast<uint4*>(a.o_part + (prow * a.k + slot) * (int64_t)a.H_q * DH) + h;
+            // partial layout [row][slot][d_h/16][H_q][16]: the G heads of a position are adjacent
+            // 32-byte units, so each warp-wide 32-byte store writes contiguous runs (half as many store
+            // instructions as 16-byte units would take for the same bytes)
+            uint32_t* d8 = reinterpret_cast<uint32_t*>(a.o_part + (prow * a.k + slot) * (int64_t)a.H_q * DH) + h * 8;
             const uint64_t il2 = f2_pack(inv_l, inv_l);
             // the whole output row is read (64-column halves, converted to bf16 as they arrive) before
             // any store, and the region is released to the next PV right after the last read
@@ -639,10 +640,15 @@ __global__ void __launch_bounds__(512, 1)
                     w[hf * 32 + z] = pack_bf16x2(f2_lo(y), f2_hi(y));
                 }
             }
+            // Stores paced ~32 ns apart: issued back to back, the four epilogue warps' 32 KB backs up
+            // the SM's memory pipeline and delays the MMA completion signals queued behind it (S(t)
+            // was seen by the softmax ~5000 clk after its last MMA, ~300 clk with the pacing)
             if (store) {
 #pragma unroll
-                for (int u = 0; u < DH / 8; ++u)
-                    d4[u * a.H_q] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                for (int u = 0; u < DH / 16; ++u) {
+                    st_global_v8(d8 + (int64_t)u * a.H_q * 8, w + 8 * u);
+                    if (u + 1 < DH / 16) __nanosleep(32);
+                }
             }
             if (store) a.lse_part[(prow * a.k + slot) * a.H_q + h] = lse_row;
             if (row == 0) TL(7, qt);
