@@ -138,6 +138,22 @@ def reference_arm(args, rank):
             times.append(dt)
             rows_done.append(len(rows))
     value = sum(rows_done) / sum(times)
+    dec = None
+    if not args.no_decode:
+        # decode: the first sequences of the decode workload (the same caches the GPU arm builds), timed
+        # as one oracle decode call per step
+        dfull = synth.DECODE_CONFIGS[args.decode_workload]
+        dcfg = dfull.with_(B=4)
+        dinp = synth.decode_inputs(dcfg, lens=synth.decode_lens(dfull)[: dcfg.B])
+        dts = []
+        for s in range(1 + args.steps):
+            t0 = time.perf_counter()
+            o.decode(dinp, dcfg.B_k, dcfg.k)
+            if s >= 1:
+                dts.append(time.perf_counter() - t0)
+        dec = {"value": dcfg.B * len(dts) / sum(dts), "unit": "tokens/s", "ms_per_step": 1000 * statistics.mean(dts),
+               "sample": f"{dcfg.B} sequences of {dfull.name} (cache lengths {dinp['lens'].tolist()}), "
+                         "one decode token each: block pooling, Top-k and sparse attention, fp64"}
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -148,6 +164,8 @@ def reference_arm(args, rank):
                              "sample": f"per step {rows_done[0]} sampled query rows of {cfg.name} "
                                        "(selection + attention, all heads)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if dec is not None:
+        line["decode"] = dec
     print(json.dumps(line), flush=True)
 
 
