@@ -4,9 +4,10 @@
 // Sequence beta's query sits at position i = len - 1; its selection and attention are those of
 // prefill row i (explainer Figure 1 and section 05). Three kernels, then the shared combine:
 //   1. decode_pool   : index scores q_idx . k_idx over the whole k_idx cache, block max-pooled.
-//                      HBM-bound streaming (~len*H_kv*d_idx*2 bytes per sequence), CUDA cores: one
-//                      warp reads a 512-byte cache row per load, each lane dots 8 elements, lanes of a
-//                      group reduce with shuffles. Exact for integer-valued index inputs.
+//                      HBM-bound streaming (~len*H_kv*d_idx*2 bytes per sequence): whole cache blocks
+//                      by bulk copy into a 3-stage shared-memory ring per SM, scored on CUDA cores (a
+//                      warp-wide load covers whole cache rows, each lane dots 8 elements, lanes of a
+//                      group reduce with shuffles). Exact for integer-valued index inputs.
 //   2. decode_topk   : per (sequence, group) one warp; each lane keeps a register Top-(k-1) list over
 //                      its 1/32 of the pooled row, then a warp-shuffle merge (explainer section 05-1)
 //                      and the forced local block.
@@ -25,8 +26,16 @@ namespace msa {
 
 namespace {
 
-constexpr int kPoolWarps = 8;
-constexpr int kPoolCtasPerSm = 8;
+constexpr int kPoolConsumers = 8;                  // scoring warps of a pooling CTA
+constexpr int kPoolStages = 3;                     // k_idx cache blocks in flight per SM
+constexpr int kPoolStageBytes = kBk * 512;         // one block of rows up to 512 bytes (H_kv * d_idx <= 256)
+
+struct PoolShared {
+    uint64_t full[kPoolStages], empty[kPoolStages];
+    float pmax[kPoolStages][kPoolConsumers][32]; // [stage][warp][group]: the warp's rows' maximum
+    int abort_flag;
+};
+constexpr int kPoolSmem = kPoolStages * kPoolStageBytes + (int)sizeof(PoolShared);
 
 __device__ __forceinline__ int seq_local_block(int len) { return (len - 1) / kBk; }
 
@@ -75,37 +84,99 @@ __global__ void __launch_bounds__(1024) decode_prefix_kernel(DecodeArgs a)
     }
 }
 
-__global__ void __launch_bounds__(kPoolWarps * 32) decode_pool_kernel(DecodeArgs a, int nb_max)
+// One CTA per SM streams an equal contiguous slice of the flattened block list. Its producer thread
+// keeps kPoolStages whole blocks of the k_idx cache in flight (one bulk copy each: a block's 128 rows
+// are contiguous), and kPoolConsumers warps score 128 / kPoolConsumers rows of every block from
+// shared memory: a warp-wide 16-byte load per lane covers whole cache rows, each lane dots its 8
+// elements, the lanes of a group reduce by shuffles. Each warp leaves its per-group maxima in shared
+// memory; the producer reduces them and writes the pooled scores before it refills the stage.
+__global__ void __launch_bounds__((kPoolConsumers + 1) * 32, 1) decode_pool_kernel(DecodeArgs a, int nb_max)
 {
+    extern __shared__ __align__(1024) uint8_t pool_smem[];
+    PoolShared& sh = *reinterpret_cast<PoolShared*>(pool_smem + kPoolStages * kPoolStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int lanes_per_pos = (a.H_kv * a.d_idx) / 8;
-    const int pos_per_step = 32 / lanes_per_pos;
-    const int lanes_per_group = a.d_idx / 8;
-    const int sub = lane % lanes_per_pos;
-    const int r = sub / lanes_per_group;
-    const int pos_lane = lane / lanes_per_pos;
     const int64_t row_elems = (int64_t)a.H_kv * a.d_idx;
+    const uint32_t blk_bytes = (uint32_t)(kBk * row_elems * 2);
     const int64_t total = a.blk_prefix[a.B];
-    const int64_t n_warps = (int64_t)gridDim.x * kPoolWarps;
-    const int64_t wid = (int64_t)blockIdx.x * kPoolWarps + warp;
-    const int64_t g0 = total * wid / n_warps, g1 = total * (wid + 1) / n_warps;
+    const int64_t g0 = total * blockIdx.x / gridDim.x, g1 = total * (blockIdx.x + 1) / gridDim.x;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kPoolStages; ++i) {
+            mbar_init(&sh.full[i], 1);
+            mbar_init(&sh.empty[i], kPoolConsumers);
+        }
+        sh.abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
     if (g0 >= g1) return;
+    volatile int* abort_flag = &sh.abort_flag;
     // the sequence holding block g0: the last beta with prefix[beta] <= g0
     int lo = 0, hi = a.B - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (a.blk_prefix[mid] <= g0) lo = mid; else hi = mid - 1;
     }
-    int beta = -1;
-    int64_t seq_begin = 0, seq_end = 0;
-    float qf[8];
-    const uint16_t* cache = nullptr;
-    for (int64_t g = g0; g < g1; ++g) {
-        if (g >= seq_end) { // enter the next sequence that owns blocks (empty ones are skipped)
-            beta = beta < 0 ? lo : beta + 1;
+    if (warp == kPoolConsumers) {
+        // ---------------------------------------------------------------- producer (lane 0)
+        if (lane != 0) return;
+        int pend_beta[kPoolStages], pend_b[kPoolStages];
+        auto flush = [&](int s) { // all consumers are done with stage s: its block's pooled scores
+            for (int r = 0; r < a.H_kv; ++r) {
+                float m = sh.pmax[s][0][r];
+#pragma unroll
+                for (int w = 1; w < kPoolConsumers; ++w) m = fmaxf(m, sh.pmax[s][w][r]);
+                a.pooled[((int64_t)pend_beta[s] * a.H_kv + r) * nb_max + pend_b[s]] = m;
+            }
+        };
+        int beta = lo;
+        bool ok = true;
+        int64_t n = 0;
+        for (int64_t g = g0; g < g1; ++g, ++n) {
+            const int s = (int)(n % kPoolStages);
+            if (n >= kPoolStages) {
+                if (!wait_or_abort(&sh.empty[s], (uint32_t)((n / kPoolStages - 1) & 1), abort_flag, a.err, 50,
+                                   kWaitLimit)) {
+                    ok = false;
+                    break;
+                }
+                flush(s);
+            }
             while (a.blk_prefix[beta + 1] <= g) ++beta;
-            seq_begin = a.blk_prefix[beta];
-            seq_end = a.blk_prefix[beta + 1];
+            const int b = (int)(g - a.blk_prefix[beta]);
+            pend_beta[s] = beta;
+            pend_b[s] = b;
+            mbar_arrive_expect_tx(&sh.full[s], blk_bytes);
+            bulk_load(pool_smem + s * kPoolStageBytes,
+                      a.k_idx_cache + ((int64_t)beta * a.L_max + (int64_t)b * kBk) * row_elems, blk_bytes,
+                      &sh.full[s]);
+        }
+        // the last stages: flush them, or (after an abort) wait for their copies before the CTA exits
+        for (int64_t m = n > kPoolStages ? n - kPoolStages : 0; m < n; ++m) {
+            const int s = (int)(m % kPoolStages);
+            if (ok && wait_or_abort(&sh.empty[s], (uint32_t)((m / kPoolStages) & 1), abort_flag, a.err, 51,
+                                    kWaitLimit))
+                flush(s);
+            else
+                drain_wait(&sh.full[s], (uint32_t)((m / kPoolStages) & 1), a.err, 52, kWaitLimit);
+        }
+        return;
+    }
+    // -------------------------------------------------------------------- consumers
+    const int lanes_per_pos = (int)(row_elems / 8);
+    const int pos_per_step = 32 / lanes_per_pos;
+    const int lanes_per_group = a.d_idx / 8;
+    const int sub = lane % lanes_per_pos;
+    const int r = sub / lanes_per_group;
+    const int pos_lane = lane / lanes_per_pos;
+    constexpr int kRows = kBk / kPoolConsumers; // rows of every block this warp scores
+    int beta = lo - 1;
+    float qf[8];
+    int64_t n = 0;
+    for (int64_t g = g0; g < g1; ++g, ++n) {
+        const int s = (int)(n % kPoolStages);
+        if (beta < lo || a.blk_prefix[beta + 1] <= g) { // entering the next sequence that owns blocks
+            beta = beta < lo ? lo : beta + 1;
+            while (a.blk_prefix[beta + 1] <= g) ++beta;
             const uint4 qv = *reinterpret_cast<const uint4*>(a.q_idx + ((int64_t)beta * a.H_kv) * a.d_idx + sub * 8);
             const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
@@ -113,21 +184,19 @@ __global__ void __launch_bounds__(kPoolWarps * 32) decode_pool_kernel(DecodeArgs
                 qf[2 * q] = __uint_as_float(qw[q] << 16);
                 qf[2 * q + 1] = __uint_as_float(qw[q] & 0xFFFF0000u);
             }
-            cache = a.k_idx_cache + (int64_t)beta * a.L_max * row_elems + sub * 8;
         }
-        const int b = (int)(g - seq_begin);
+        if (!wait_or_abort(&sh.full[s], (uint32_t)((n / kPoolStages) & 1), abort_flag, a.err, 53, kWaitLimit)) break;
+        const uint16_t* blk = reinterpret_cast<const uint16_t*>(pool_smem + s * kPoolStageBytes) + sub * 8;
         float m = -CUDART_INF_F;
-        const uint16_t* blk = cache + (int64_t)b * kBk * row_elems;
-        // 8 cache rows in flight per warp: issue the loads, then reduce
-        for (int j0 = 0; j0 < kBk; j0 += 8 * pos_per_step) {
+        for (int j0 = 0; j0 < kRows; j0 += 8 * pos_per_step) {
             uint4 kv[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int j = j0 + u * pos_per_step + pos_lane;
-                kv[u] = j < kBk ? __ldg(reinterpret_cast<const uint4*>(blk + (int64_t)j * row_elems))
-                                : make_uint4(0u, 0u, 0u, 0u);
+                kv[u] = j < kRows ? *reinterpret_cast<const uint4*>(blk + (int64_t)(warp * kRows + j) * row_elems)
+                                  : make_uint4(0u, 0u, 0u, 0u);
             }
-            float s[8];
+            float sc[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const uint32_t kw[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
@@ -137,19 +206,20 @@ __global__ void __launch_bounds__(kPoolWarps * 32) decode_pool_kernel(DecodeArgs
                     acc = fmaf(qf[2 * q], __uint_as_float(kw[q] << 16), acc);
                     acc = fmaf(qf[2 * q + 1], __uint_as_float(kw[q] & 0xFFFF0000u), acc);
                 }
-                s[u] = acc;
+                sc[u] = acc;
             }
             for (int o = lanes_per_group >> 1; o > 0; o >>= 1) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
+                for (int u = 0; u < 8; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                if (j0 + u * pos_per_step < kBk) m = fmaxf(m, s[u]);
+                if (j0 + u * pos_per_step < kRows) m = fmaxf(m, sc[u]);
         }
         for (int o = lanes_per_pos; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane < lanes_per_pos && (sub % lanes_per_group) == 0)
-            a.pooled[((int64_t)beta * a.H_kv + r) * nb_max + b] = m;
+        if (lane < lanes_per_pos && (sub % lanes_per_group) == 0) sh.pmax[s][warp][r] = m;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
     }
 }
 
@@ -398,17 +468,16 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(DecodeArgs a)
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s)
 {
     const int nb_max = (int)((a.L_max + kBk - 1) / kBk);
-    int dev = 0, n_sm = 148, per_sm = 0;
+    int dev = 0, n_sm = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-    // one wave of resident CTAs: every warp gets an equal slice, so a second wave would only add a tail
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_pool_kernel, kPoolWarps * 32, 0) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
-    if (per_sm > kPoolCtasPerSm) per_sm = kPoolCtasPerSm;
+    if (a.H_kv * a.d_idx > 256) return cudaErrorInvalidValue; // a cache row must fit a 512-byte stage row
+    cudaError_t e0 = cudaFuncSetAttribute(decode_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPoolSmem);
+    if (e0 != cudaSuccess) return e0;
     trace_begin(s);
     decode_prefix_kernel<<<1, 1024, 0, s>>>(a);
-    decode_pool_kernel<<<n_sm * per_sm, kPoolWarps * 32, 0, s>>>(a, nb_max);
+    // one CTA per SM, each an equal slice of the flattened block list
+    decode_pool_kernel<<<n_sm, (kPoolConsumers + 1) * 32, kPoolSmem, s>>>(a, nb_max);
     trace_end(s, MSA_KERNEL_DEC_POOL);
     trace_begin(s);
     decode_topk_kernel<<<dim3(a.B, a.H_kv), 32, 0, s>>>(a, nb_max);
