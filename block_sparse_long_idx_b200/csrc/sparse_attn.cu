@@ -117,7 +117,7 @@ struct AttnShared {
 
 constexpr uint32_t kNegInfBits = 0xff800000u;
 constexpr int REG_LAUNCH = 128; // 65536 registers / 512 threads
-constexpr int REG_PRODUCER = 96, REG_SOFTMAX = 128, REG_EPILOGUE = 160;
+constexpr int REG_PRODUCER = 80, REG_SOFTMAX = 128, REG_EPILOGUE = 176;
 static_assert(REG_PRODUCER + 2 * REG_SOFTMAX + REG_EPILOGUE <= 4 * REG_LAUNCH, "register split exceeds the launch budget");
 
 __device__ __forceinline__ uint32_t a_col(int t) { return (uint32_t)(t % kRegions) * 128; }
@@ -615,30 +615,28 @@ __global__ void __launch_bounds__(512, 1)
             // instructions as 16-byte units would take for the same bytes)
             uint32_t* d8 = reinterpret_cast<uint32_t*>(a.o_part + (prow * a.k + slot) * (int64_t)a.H_q * DH) + h * 8;
             const uint64_t il2 = f2_pack(inv_l, inv_l);
-            // the whole output row is read (64-column halves, converted to bf16 as they arrive) before
-            // any store, and the region is released to the next PV right after the last read
-            uint32_t w[DH / 2];
+            // the whole output row is read with one wait and the region released to the next PV before
+            // any conversion; the bf16 pairs are then packed in place (word z from words 2z, 2z+1)
+            uint32_t w[DH];
+            tmem_ld32_at<0>(lane_base + kOCol, w);
+            tmem_ld32_at<32>(lane_base + kOCol + 32, w);
+            if constexpr (DH > 64) {
+                tmem_ld32_at<64>(lane_base + kOCol + 64, w);
+                tmem_ld32_at<96>(lane_base + kOCol + 96, w);
+            }
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sh.o_free);
+                mbar_arrive(&sh.tile_free[rs]); // S, softmax and PV of qt are done with the record
+                TL(24 + quarter, qt);
+            }
+            if (row == 0) TL(13, qt);
 #pragma unroll
-            for (int hf = 0; hf < DH / 64; ++hf) {
-                uint32_t o[64];
-                tmem_ld32_at<0>(lane_base + kOCol + hf * 64, o);
-                tmem_ld32_at<32>(lane_base + kOCol + hf * 64 + 32, o);
-                tmem_ld_wait();
-                if (hf == DH / 64 - 1) { // O fully read: the next tile's PV may overwrite it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&sh.o_free);
-                        mbar_arrive(&sh.tile_free[rs]); // S, softmax and PV of qt are done with the record
-                        TL(24 + quarter, qt);
-                    }
-                    if (row == 0) TL(13, qt);
-                }
-#pragma unroll
-                for (int z = 0; z < 32; ++z) {
-                    const uint64_t y = f2_mul(f2_pack(__uint_as_float(o[2 * z]), __uint_as_float(o[2 * z + 1])), il2);
-                    w[hf * 32 + z] = pack_bf16x2(f2_lo(y), f2_hi(y));
-                }
+            for (int z = 0; z < DH / 2; ++z) {
+                const uint64_t y = f2_mul(f2_pack(__uint_as_float(w[2 * z]), __uint_as_float(w[2 * z + 1])), il2);
+                w[z] = pack_bf16x2(f2_lo(y), f2_hi(y));
             }
             // Stores paced ~32 ns apart: issued back to back, the four epilogue warps' 32 KB backs up
             // the SM's memory pipeline and delays the MMA completion signals queued behind it (S(t)
