@@ -70,14 +70,14 @@ def load_peaks():
 # full launch is the per-row figure times its rows. A figure only applies to the kernel source it was
 # measured on (the kernel's own .cu file, by hash): after any change to it the bench reports null.
 PROFILED_TRAFFIC = {
-    "attn": {"files": ("sparse_attn.cu",), "sha256_16": "cd81b9df8683b0b0",
-             "bytes_per_row": (382.179072e6 + 2.123139e9) / 8192,
+    "attn": {"files": ("sparse_attn.cu",), "sha256_16": "b3f4e84dc09c6d39",
+             "bytes_per_row": (379.072e6 + 2.124692e9) / 8192,
              "capture": "ncu capture of sparse_attn_kernel<128, 16, 0> on the N=32768 prefill, one 8192-row pass"},
-    "attn_fp8": {"files": ("sparse_attn.cu",), "sha256_16": "cd81b9df8683b0b0",
-                 "bytes_per_row": (224.727808e6 + 2.123034e9) / 8192,
+    "attn_fp8": {"files": ("sparse_attn.cu",), "sha256_16": "b3f4e84dc09c6d39",
+                 "bytes_per_row": (228.76288e6 + 2.123282e9) / 8192,
                  "capture": "ncu capture of sparse_attn_kernel<128, 16, 1> on the N=32768 prefill, one 8192-row pass"},
-    "combine": {"files": ("combine.cu",), "sha256_16": "8436940a71c651a1",
-                "bytes_per_row": 282506.7,
+    "combine": {"files": ("combine.cu",), "sha256_16": "c171e6105a4b5769",
+                "bytes_per_row": (2.181085e9 + 132.157184e6) / 8192,
                 "capture": "ncu capture of combine_kernel on the N=32768 prefill, one 8192-row pass"},
 }
 
